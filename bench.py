@@ -1,0 +1,486 @@
+#!/usr/bin/env python
+"""Benchmark of the exact tiled attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  * prefill: causal MHA bf16, B=4, Hq=Hkv=16, N=2048, d=128 (O and LSE);
+  * decode:  GQA bf16, 64 sequences, Hq=32, Hkv=8, d=128, KV lengths uniform
+             in [1024, 8192] (split-KV pass + LSE combine).
+`value` is the prefill throughput in TFLOP/s (algorithmic FLOPs: 4*d per
+visible query/key pair) over the prefill kernel's CUDA-event time, summed over
+ranks (weak scaling: every rank runs its own batch). The decode side is
+reported in the `decode` object in GB/s of KV cache read. L2 is flushed (a
+256 MiB write) before every step; the flush is outside the kernel events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With --impl reference the fp64 CPU oracle runs a bounded sample of the same
+workload on the host cores (rank 0 only) and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s & decode KV-cache GB/s, as % of B200 roofline"
+PREFILL = workloads.PREFILL_MHA_2K
+DECODE = workloads.DECODE_GQA_RAGGED
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = [
+    os.path.join(ROOT, "exact_tiled_attention_38_b200", "csrc", f)
+    for f in ("prefill_sm100.cuh", "decode_sm100.cuh", "common.cuh", "ptx.cuh")
+]
+
+
+# ----------------------------------------------------------------------------- accounting
+def visible_pairs(nq: int, nk: int, causal: bool) -> int:
+    """(query, key) pairs a row-wise softmax sees; causal is bottom-right aligned."""
+    if not causal:
+        return nq * nk
+    per_row = np.clip(np.arange(nq, dtype=np.int64) + (nk - nq) + 1, 0, nk)
+    return int(per_row.sum())
+
+
+def prefill_flops(w) -> float:
+    return 4.0 * w.d * w.B * w.Hq * visible_pairs(w.Nq, w.Nk, w.causal)
+
+
+def decode_kv_bytes(seqlens, Hkv: int, d: int, elem: int = 2) -> int:
+    total = int(np.clip(np.asarray(seqlens, dtype=np.int64), 0, None).sum())
+    return 2 * total * Hkv * d * elem
+
+
+def decode_bytes(seqlens, B, Hq, Hkv, d, elem=2) -> int:
+    """Algorithmic HBM bytes of one decode call: KV read + q read + O/LSE write."""
+    return decode_kv_bytes(seqlens, Hkv, d, elem) + 2 * B * Hq * d * elem + B * Hq * 4
+
+
+def prefill_bytes(w) -> int:
+    e = 2
+    q = w.B * w.Hq * w.Nq * w.d * e
+    kv = 2 * w.B * w.Hkv * w.Nk * w.d * e
+    return 2 * q + kv + w.B * w.Hq * w.Nq * 4
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source
+    has not changed since it was captured; else None."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = d.get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return world, rank, local
+
+
+def reduce_max(values, group=None):
+    """Element-wise max over ranks of a list of floats (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    backend = dist.get_backend(group)
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else "cpu"
+    t = torch.tensor(list(values), dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return t.cpu().tolist()
+
+
+def aggregate_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: units all ranks processed / slowest rank's time (per s)."""
+    return units_per_rank * world / (max_ms * 1e-3)
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while the timed loop runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(
+                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                    timeout=5).stdout.strip()
+                if out:
+                    self.rows.append([x.strip() for x in out.split(",")])
+            except Exception:
+                return
+            self._stop.wait(0.1)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if len(r) > 5 + i and r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = threadpool_info()
+        n = [i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_prefill_sample(q, k, v, heads):
+    """fp64 oracle on `heads` (b, h) pairs of the prefill workload. Returns seconds."""
+    import oracle
+
+    t0 = time.perf_counter()
+    for b, h in heads:
+        g = h // (PREFILL.Hq // PREFILL.Hkv)
+        oracle.attention_ref(q[b:b + 1, h:h + 1], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1],
+                             PREFILL.scale, PREFILL.causal)
+    return time.perf_counter() - t0
+
+
+def oracle_decode_sample(q, kc, vc, sl, seqs):
+    import oracle
+
+    t0 = time.perf_counter()
+    lens = sl.tolist()
+    offs = np.concatenate([[0], np.cumsum(lens)])
+    per = DECODE.Hkv * DECODE.d
+    for b in seqs:
+        a, e = int(offs[b]) * per, int(offs[b + 1]) * per
+        oracle.decode_ref(q[b:b + 1], kc[a:e], vc[a:e], sl[b:b + 1], DECODE.scale, DECODE.Hkv)
+    return time.perf_counter() - t0
+
+
+def cpu_inputs():
+    """Host copies of a slice of the workload for the oracle (CPU generators)."""
+    import torch
+
+    q, k, v = workloads.prefill_inputs(PREFILL, device="cpu")
+    dq, dkc, dvc, dsl = workloads.decode_inputs(DECODE, device="cpu")
+    return (q, k, v), (dq, dkc, dvc, dsl)
+
+
+def cpu_baseline(budget_s: float = 12.0):
+    """Time the oracle, as it stands, on a bounded sample of the workload."""
+    (q, k, v), (dq, dkc, dvc, dsl) = cpu_inputs()
+    flops_head = prefill_flops(PREFILL) / (PREFILL.B * PREFILL.Hq)
+    heads, spent = [], 0.0
+    order = [(b, h) for b in range(PREFILL.B) for h in range(PREFILL.Hq)]
+    while spent < budget_s / 2 and len(heads) < len(order):
+        hb = order[len(heads)]
+        spent += oracle_prefill_sample(q, k, v, [hb])
+        heads.append(hb)
+    p_tflops = flops_head * len(heads) / spent / 1e12
+    seqs, dspent = [], 0.0
+    while dspent < budget_s / 2 and len(seqs) < DECODE.B:
+        dspent += oracle_decode_sample(dq, dkc, dvc, dsl, [len(seqs)])
+        seqs.append(len(seqs))
+    kv = decode_kv_bytes(dsl[: len(seqs)].numpy(), DECODE.Hkv, DECODE.d)
+    d_gbs = kv / dspent / 1e9
+    return {
+        "value": p_tflops, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+        "sample": f"prefill: {len(heads)} of {PREFILL.B * PREFILL.Hq} (b,h) heads of "
+                  f"{PREFILL.name} in {spent:.1f} s; decode: {len(seqs)} of {DECODE.B} "
+                  f"sequences of {DECODE.name} in {dspent:.1f} s",
+        "decode": {"value": d_gbs, "unit": "GB/s"},
+    }
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    (q, k, v), (dq, dkc, dvc, dsl) = cpu_inputs()
+    flops_head = prefill_flops(PREFILL) / (PREFILL.B * PREFILL.Hq)
+    order = [(b, h) for b in range(PREFILL.B) for h in range(PREFILL.Hq)]
+    for i in range(args.warmup):
+        oracle_prefill_sample(q, k, v, [order[i % len(order)]])
+    pt = dt = 0.0
+    kv = 0
+    for i in range(args.steps):
+        pt += oracle_prefill_sample(q, k, v, [order[i % len(order)]])
+        b = i % DECODE.B
+        dt += oracle_decode_sample(dq, dkc, dvc, dsl, [b])
+        kv += decode_kv_bytes(dsl[b:b + 1].numpy(), DECODE.Hkv, DECODE.d)
+    value = flops_head * args.steps / pt / 1e12
+    sample = (f"each step: 1 of {PREFILL.B * PREFILL.Hq} (b,h) heads of {PREFILL.name} and 1 of "
+              f"{DECODE.B} sequences of {DECODE.name}, fp64 numpy")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": (pt + dt) / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{PREFILL.name} + {DECODE.name} (bounded sample per step)",
+                   "parallelism": "rank 0 host cores"},
+        "decode": {"value": kv / dt / 1e9, "unit": "GB/s"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    import exact_tiled_attention_38_b200 as eta
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    eta.load_library()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    seed_off = 1000 * rank
+    q, k, v = workloads.prefill_inputs(PREFILL, device=dev, seed=PREFILL.seed + seed_off)
+    o = torch.empty_like(q)
+    lse = torch.empty(PREFILL.B, PREFILL.Hq, PREFILL.Nq, device=dev, dtype=torch.float32)
+    sl_cpu = workloads.decode_seqlens(DECODE.B, DECODE.lmin, DECODE.lmax,
+                                      DECODE.seed + seed_off)
+    dq, dkc, dvc, dsl = workloads.decode_inputs(DECODE, device=dev, seqlens=sl_cpu,
+                                                seed=DECODE.seed + seed_off)
+    do = torch.empty_like(dq)
+    dlse = torch.empty(DECODE.B, DECODE.Hq, device=dev, dtype=torch.float32)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)  # 256 MiB > L2
+
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        flush.zero_()
+        if evs:
+            evs[0].record(stream)
+        eta.attn_fwd(q, k, v, o=o, lse=lse, scale=PREFILL.scale, causal=True, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        eta.attn_decode(dq, dkc, dvc, dsl, DECODE.Hkv, o=do, lse=dlse, scale=DECODE.scale,
+                        stream=stream)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    code, raw = eta.attn_get_device_status(stream)
+    if code != eta.ATTN_OK:
+        raise RuntimeError(f"device status {code} ({raw:#x}) after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    code, raw = eta.attn_get_device_status(stream)
+    if code != eta.ATTN_OK:
+        raise RuntimeError(f"device status {code} ({raw:#x}) in the timed loop")
+
+    pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    step_ms = t_start.elapsed_time(t_end) / args.steps
+    pre_ms_max, dec_ms_max, step_ms_max = reduce_max([pre_ms, dec_ms, step_ms])
+
+    # ---- end to end through the public API, host buffers in pinned memory
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hdq, hdkc, hdvc, hdsl = (t.cpu().pin_memory() for t in (dq, dkc, dvc, dsl))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    hdo = torch.empty(do.shape, dtype=do.dtype).pin_memory()
+    hdlse = torch.empty(dlse.shape, dtype=dlse.dtype).pin_memory()
+    bufs = [torch.empty_like(t) for t in (q, k, v, dq, dkc, dvc, dsl)]
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hdkc, hdvc, hdsl))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdo, hdlse))
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        for dst, src in zip(bufs[:3], (hq, hk, hv)):
+            dst.copy_(src, non_blocking=True)
+        oo, ll = eta.attn_fwd(bufs[0], bufs[1], bufs[2], scale=PREFILL.scale, causal=True,
+                              stream=stream)
+        ho.copy_(oo, non_blocking=True)
+        hlse.copy_(ll, non_blocking=True)
+        if ev:
+            ev[1].record(stream)
+        for dst, src in zip(bufs[3:], (hdq, hdkc, hdvc, hdsl)):
+            dst.copy_(src, non_blocking=True)
+        oo, ll = eta.attn_decode(bufs[3], bufs[4], bufs[5], bufs[6], DECODE.Hkv,
+                                 scale=DECODE.scale, stream=stream)
+        hdo.copy_(oo, non_blocking=True)
+        hdlse.copy_(ll, non_blocking=True)
+        if ev:
+            ev[2].record(stream)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    eev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(e2e_steps)]
+    if world > 1:
+        dist.barrier()
+    for i in range(e2e_steps):
+        e2e_step(eev[i])
+    torch.cuda.synchronize()
+    e2e_pre = sum(e[0].elapsed_time(e[1]) for e in eev) / e2e_steps
+    e2e_dec = sum(e[1].elapsed_time(e[2]) for e in eev) / e2e_steps
+    e2e_pre, e2e_dec = reduce_max([e2e_pre, e2e_dec])
+
+    flops = prefill_flops(PREFILL)
+    kv_bytes = decode_kv_bytes(sl_cpu.numpy(), DECODE.Hkv, DECODE.d)
+    dbytes = decode_bytes(sl_cpu.numpy(), DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.d)
+    value = aggregate_throughput(flops, world, pre_ms_max) / 1e12
+    dec_gbs = aggregate_throughput(kv_bytes, world, dec_ms_max) / 1e9
+    peaks, src = load_peaks()
+    pre_ach = flops / (pre_ms * 1e-3) / 1e12
+    dec_ach = dbytes / (dec_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{PREFILL.name} + {DECODE.name}",
+            "prefill": {"B": PREFILL.B, "Hq": PREFILL.Hq, "Hkv": PREFILL.Hkv, "N": PREFILL.Nq,
+                        "d": PREFILL.d, "causal": True, "flops": flops},
+            "decode": {"B": DECODE.B, "Hq": DECODE.Hq, "Hkv": DECODE.Hkv, "d": DECODE.d,
+                       "kv_tokens": int(sl_cpu.sum()), "kv_bytes": kv_bytes,
+                       "nsplit": eta.attn_decode_num_splits(DECODE.B, DECODE.Hq, DECODE.Hkv,
+                                                            DECODE.d)},
+            "l2": "flushed before every step (256 MiB write, outside the kernel events)",
+            "parallelism": f"replicas x{world} (independent batches per GPU)",
+        },
+        "roofline": {"bound": "tensor", "achieved": pre_ach, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": pre_ach / peaks["bf16_tflops"],
+                     "traffic": profiled_traffic("attn_prefill_kernel"),
+                     "kernel": "attn_prefill_kernel<128,bf16,causal>",
+                     "peak_source": f"{src} bf16 burst",
+                     "ms_per_launch": pre_ms},
+        "decode": {
+            "value": dec_gbs, "unit": "GB/s (KV cache read)", "ms_per_call": dec_ms,
+            "roofline": {"bound": "hbm", "achieved": dec_ach, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": dec_ach / peaks["hbm_gbs"],
+                         "traffic": profiled_traffic("attn_decode_split_kernel"),
+                         "kernel": "attn_decode_split_kernel<128,4,bf16> + combine",
+                         "peak_source": f"{src} copy bandwidth"},
+        },
+        "e2e": {"value": aggregate_throughput(flops, world, e2e_pre) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "decode_gbs": aggregate_throughput(kv_bytes, world, e2e_dec) / 1e9,
+                "steps": e2e_steps},
+        "clocks": clocks.summary(),
+        "gpu_launches": 3 * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

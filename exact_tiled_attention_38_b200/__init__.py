@@ -1,0 +1,198 @@
+"""Python binding for the exact tiled attention library (``include/attn.h``).
+
+Argument marshalling only: every function checks shapes and dtypes of torch
+tensors, then calls the C entry point of the same name with raw device
+pointers and the current CUDA stream. All arithmetic runs in the CUDA kernels
+of ``libattn.so``; there is no fallback path. If the library is missing or
+cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID = -1
+ATTN_ERR_UNSUPPORTED = -2
+ATTN_ERR_CUDA = -3
+ATTN_ERR_TIMEOUT = -4
+
+# name -> (restype, argtypes); mirrors include/attn.h
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+SIGNATURES = {
+    "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_fwd_f16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
+    "attn_decode_f16": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
+    "attn_decode_num_splits": (_I, [_I, _I, _I, _I]),
+    "attn_strerror": (ctypes.c_char_p, [_I]),
+    "attn_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
+}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} (code {code})")
+
+
+def load_library(path: str = LIB_PATH):
+    """Load ``libattn.so`` (once). Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is not built; run `python -m exact_tiled_attention_38_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def strerror(code: int) -> str:
+    return load_library().attn_strerror(int(code)).decode()
+
+
+def _stream_handle(stream) -> Optional[int]:
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return stream or None
+    return stream.cuda_stream or None
+
+
+def _check(code: int, where: str):
+    if code != ATTN_OK:
+        raise AttnError(code, where)
+
+
+def _dev(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _fwd(fname, dtype, q, k, v, o, lse, scale, causal, stream, want_lse):
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+        if t.dtype != dtype or t.dim() != 4:
+            raise ValueError(f"{n} must be a 4-D {dtype} tensor [B, H, N, d]")
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if Bk != B or dk != d or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q/k/v shapes disagree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    _dev(o, "o")
+    if o.dtype != dtype or tuple(o.shape) != tuple(q.shape):
+        raise ValueError("o must match q")
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32)
+    if lse is not None:
+        _dev(lse, "lse")
+        if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Nq):
+            raise ValueError("lse must be float32 [B, Hq, Nq]")
+    fn = getattr(load_library(), fname)
+    code = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+              lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
+              float(scale), 1 if causal else 0, _stream_handle(stream))
+    _check(code, fname)
+    return o, lse
+
+
+def attn_fwd(q, k, v, o=None, lse=None, scale: Optional[float] = None, causal: bool = False,
+             stream=None, want_lse: bool = True) -> Tuple:
+    """Prefill attention, bf16. q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] -> (o, lse)."""
+    import torch
+
+    return _fwd("attn_fwd", torch.bfloat16, q, k, v, o, lse, scale, causal, stream, want_lse)
+
+
+def attn_fwd_f16(q, k, v, o=None, lse=None, scale: Optional[float] = None,
+                 causal: bool = False, stream=None, want_lse: bool = True) -> Tuple:
+    """Prefill attention, fp16."""
+    import torch
+
+    return _fwd("attn_fwd_f16", torch.float16, q, k, v, o, lse, scale, causal, stream,
+                want_lse)
+
+
+def _decode(fname, dtype, q, kcache, vcache, seqlens, Hkv, o, lse, scale, stream, want_lse):
+    import torch
+
+    for t, n in ((q, "q"), (kcache, "kcache"), (vcache, "vcache"), (seqlens, "seqlens")):
+        _dev(t, n)
+    if q.dtype != dtype or q.dim() != 3:
+        raise ValueError(f"q must be a 3-D {dtype} tensor [B, Hq, d]")
+    if kcache.dtype != dtype or vcache.dtype != dtype:
+        raise ValueError(f"caches must be {dtype}")
+    if seqlens.dtype != torch.int32:
+        raise ValueError("seqlens must be int32")
+    B, Hq, d = q.shape
+    if seqlens.numel() != B:
+        raise ValueError("seqlens must have B entries")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    _dev(o, "o")
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    fn = getattr(load_library(), fname)
+    code = fn(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
+              o.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, d,
+              float(scale), _stream_handle(stream))
+    _check(code, fname)
+    return o, lse
+
+
+def attn_decode(q, kcache, vcache, seqlens, Hkv: int, o=None, lse=None,
+                scale: Optional[float] = None, stream=None, want_lse: bool = True):
+    """One-token decode over a packed ragged cache, bf16. Returns (o [B,Hq,d], lse [B,Hq])."""
+    import torch
+
+    return _decode("attn_decode", torch.bfloat16, q, kcache, vcache, seqlens, Hkv, o, lse,
+                   scale, stream, want_lse)
+
+
+def attn_decode_f16(q, kcache, vcache, seqlens, Hkv: int, o=None, lse=None,
+                    scale: Optional[float] = None, stream=None, want_lse: bool = True):
+    """One-token decode, fp16."""
+    import torch
+
+    return _decode("attn_decode_f16", torch.float16, q, kcache, vcache, seqlens, Hkv, o, lse,
+                   scale, stream, want_lse)
+
+
+def attn_decode_num_splits(B: int, Hq: int, Hkv: int, d: int) -> int:
+    r = load_library().attn_decode_num_splits(B, Hq, Hkv, d)
+    if r < 0:
+        raise AttnError(r, "attn_decode_num_splits")
+    return r
+
+
+def attn_get_device_status(stream=None) -> Tuple[int, int]:
+    """(status code, raw site code) after synchronising the stream; clears the word."""
+    raw = ctypes.c_uint(0)
+    code = load_library().attn_get_device_status(_stream_handle(stream), ctypes.byref(raw))
+    return code, raw.value

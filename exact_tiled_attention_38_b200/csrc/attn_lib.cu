@@ -1,0 +1,334 @@
+// C-ABI boundary of the attention library: argument checks, TMA descriptor
+// encoding, launch configuration and error codes. Every step of the
+// computation runs in the kernels of prefill_sm100.cuh and decode_sm100.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+namespace eta {
+namespace api {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
+  return fn;
+}
+
+struct DeviceInfo {
+  int sm_count = 0;
+  bool sm100 = false;
+};
+
+// Per-device properties, queried once per device.
+int device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!have[dev]) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    cache[dev].sm_count = sms;
+    cache[dev].sm100 = (major == 10 && minor == 0);
+    have[dev] = true;
+  }
+  *out = cache[dev];
+  return ATTN_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+inline bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
+
+// 3-D map over a [Z][rows][D] tensor of 16-bit elements, box 64 x 128 x 1,
+// 128-byte swizzle, zero fill outside the tensor.
+int encode_3d(CUtensorMap* map, const void* base, bool bf16, int D, long long rows, long long Z) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return ATTN_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(Z)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(rows) * D * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// O = 0, LSE = -inf for `rows` rows (every row has an empty key set).
+template <typename T>
+__global__ void fill_empty_kernel(T* o, float* lse, long long rows, int D) {
+  const long long n = rows * D;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    o[i] = T(0.f);
+    if (lse != nullptr && i % D == 0) lse[i / D] = -INFINITY;
+  }
+}
+
+template <typename T>
+int launch_fill_empty(void* o, float* lse, long long rows, int D, cudaStream_t st) {
+  const long long n = rows * D;
+  const int threads = 256;
+  const long long want = (n + threads - 1) / threads;
+  const int blocks = static_cast<int>(want < 4096 ? (want > 0 ? want : 1) : 4096);
+  fill_empty_kernel<T><<<blocks, threads, 0, st>>>(reinterpret_cast<T*>(o), lse, rows, D);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, typename T, bool CAUSAL>
+int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   const prefill::Params& p, int B, cudaStream_t st) {
+  auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL>;
+  constexpr int smem = prefill::Cfg<D>::kSmemBytes;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&]() {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(B) * p.Hq, static_cast<unsigned>(p.n_pairs));
+  kern<<<grid, prefill::kThreads, smem, st>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename T>
+int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+        int Nq, int Nk, int d, float scale, int causal, cudaStream_t st, uint64_t wait_ns,
+        int debug_flags) {
+  if (B < 0 || Nq < 0 || Nk < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale))
+    return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(Nq) > 65535LL * prefill::NQT * prefill::BM) return ATTN_ERR_INVALID;
+  if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return ATTN_ERR_INVALID;
+  if (B == 0 || Nq == 0) return ATTN_OK;
+  if (o == nullptr || !aligned(o, 16) || (lse != nullptr && !aligned(lse, 4)))
+    return ATTN_ERR_INVALID;
+  if (Nk > 0 && (q == nullptr || k == nullptr || v == nullptr || !aligned(q, 16) ||
+                 !aligned(k, 16) || !aligned(v, 16)))
+    return ATTN_ERR_INVALID;
+  DeviceInfo info;
+  if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
+  if (Nk == 0) return launch_fill_empty<T>(o, lse, static_cast<long long>(B) * Hq * Nq, d, st);
+
+  constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap tq, tk, tv;
+  int rc = encode_3d(&tq, q, bf16, d, Nq, static_cast<long long>(B) * Hq);
+  if (rc == ATTN_OK) rc = encode_3d(&tk, k, bf16, d, Nk, static_cast<long long>(B) * Hkv);
+  if (rc == ATTN_OK) rc = encode_3d(&tv, v, bf16, d, Nk, static_cast<long long>(B) * Hkv);
+  if (rc != ATTN_OK) return rc;
+
+  prefill::Params p;
+  p.o = o;
+  p.lse = lse;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.n_pairs = (Nq + prefill::NQT * prefill::BM - 1) / (prefill::NQT * prefill::BM);
+  p.off = Nk - Nq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_ns = wait_ns;
+  p.debug_flags = debug_flags;
+  if (d == 128)
+    return causal ? launch_prefill<128, T, true>(tq, tk, tv, p, B, st)
+                  : launch_prefill<128, T, false>(tq, tk, tv, p, B, st);
+  return causal ? launch_prefill<64, T, true>(tq, tk, tv, p, B, st)
+                : launch_prefill<64, T, false>(tq, tk, tv, p, B, st);
+}
+
+// Split-KV count: enough CTAs for about eight waves of resident split CTAs.
+int decode_splits(int B, int Hq, int Hkv, int d, int sm_count) {
+  const int G = Hq / Hkv;
+  const int GP = G <= 4 ? 4 : 8;
+  const int nchunk = (G + GP - 1) / GP;
+  const long long units = static_cast<long long>(B) * Hkv * nchunk;
+  const int resident = (d == 128 ? 3 : 3) * sm_count;
+  long long ns = units > 0 ? (8LL * resident + units - 1) / units : 1;
+  if (ns < 1) ns = 1;
+  if (ns > 64) ns = 64;
+  return static_cast<int>(ns);
+}
+
+template <int D, int GP, typename T>
+int launch_decode_split(const decode::DParams& p, cudaStream_t st) {
+  auto kern = decode::attn_decode_split_kernel<D, GP, T>;
+  constexpr int smem = decode::DCfg<D, GP>::kSmemBytes;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&]() {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(p.Hkv * p.nchunk),
+                  static_cast<unsigned>(p.B));
+  kern<<<grid, decode::kThreads, smem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, typename T>
+int launch_decode_combine(const float* po, const float* pl, void* o, float* lse, int rows,
+                          int nsplit, cudaStream_t st) {
+  const int blocks = (rows + 3) / 4;
+  decode::attn_decode_combine_kernel<D, T>
+      <<<blocks, 128, 0, st>>>(po, pl, reinterpret_cast<T*>(o), lse, rows, nsplit);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, typename T>
+int decode_launch_all(const decode::DParams& p, void* o, float* lse, cudaStream_t st) {
+  const int GP = p.G <= 4 ? 4 : 8;
+  int rc = GP == 4 ? launch_decode_split<D, 4, T>(p, st) : launch_decode_split<D, 8, T>(p, st);
+  if (rc != ATTN_OK) return rc;
+  return launch_decode_combine<D, T>(p.part_o, p.part_lse, o, lse, p.B * p.Hq, p.nsplit, st);
+}
+
+template <typename T>
+int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* o,
+               float* lse, int B, int Hq, int Hkv, int d, float scale, cudaStream_t st) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale)) return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq > 0x7fffffffLL / 4) return ATTN_ERR_INVALID;
+  if (B == 0) return ATTN_OK;
+  if (q == nullptr || kc == nullptr || vc == nullptr || seqlens == nullptr || o == nullptr ||
+      !aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(o, 16) ||
+      !aligned(seqlens, 4) || (lse != nullptr && !aligned(lse, 4)))
+    return ATTN_ERR_INVALID;
+  DeviceInfo info;
+  if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
+
+  decode::DParams p;
+  p.q = q;
+  p.kc = kc;
+  p.vc = vc;
+  p.seqlens = seqlens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  const int GP = p.G <= 4 ? 4 : 8;
+  p.nchunk = (p.G + GP - 1) / GP;
+  p.nsplit = decode_splits(B, Hq, Hkv, d, info.sm_count);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_ns = kDefaultWaitNs;
+
+  const size_t rows = static_cast<size_t>(B) * Hq;
+  const size_t bytes = static_cast<size_t>(p.nsplit) * rows * (d + 1) * sizeof(float);
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) return ATTN_ERR_CUDA;
+  p.part_o = reinterpret_cast<float*>(ws);
+  p.part_lse = p.part_o + static_cast<size_t>(p.nsplit) * rows * d;
+  const int rc = d == 128 ? decode_launch_all<128, T>(p, o, lse, st)
+                          : decode_launch_all<64, T>(p, o, lse, st);
+  const cudaError_t fe = cudaFreeAsync(ws, st);
+  if (rc != ATTN_OK) return rc;
+  return fe == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace api
+}  // namespace eta
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, float scale, int causal, attn_stream_t stream) {
+  return eta::api::fwd<__nv_bfloat16>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                                      reinterpret_cast<cudaStream_t>(stream),
+                                      eta::kDefaultWaitNs, 0);
+}
+
+int attn_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                 int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                 attn_stream_t stream) {
+  return eta::api::fwd<__half>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                               reinterpret_cast<cudaStream_t>(stream), eta::kDefaultWaitNs, 0);
+}
+
+int attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
+                attn_stream_t stream) {
+  return eta::api::decode_run<__nv_bfloat16>(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, d,
+                                             scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_decode_f16(const void* q, const void* kcache, const void* vcache,
+                    const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv, int d,
+                    float scale, attn_stream_t stream) {
+  return eta::api::decode_run<__half>(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, d, scale,
+                                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_decode_num_splits(int B, int Hq, int Hkv, int d) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  eta::api::DeviceInfo info;
+  if (eta::api::device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
+  return eta::api::decode_splits(B, Hq, Hkv, d, info.sm_count);
+}
+
+const char* attn_strerror(int code) {
+  switch (code) {
+    case ATTN_OK:
+      return "ok";
+    case ATTN_ERR_INVALID:
+      return "invalid argument (null or misaligned pointer, bad size, Hq % Hkv != 0, or scale "
+             "not finite and > 0)";
+    case ATTN_ERR_UNSUPPORTED:
+      return "unsupported (head dim not 64 or 128, or device is not sm_100)";
+    case ATTN_ERR_CUDA:
+      return "CUDA runtime error";
+    case ATTN_ERR_TIMEOUT:
+      return "a device-side wait gave up; outputs of that launch are undefined";
+    default:
+      return "unknown error code";
+  }
+}
+
+int attn_get_device_status(attn_stream_t stream, unsigned int* raw_code) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, eta::g_status, sizeof(v)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(eta::g_status, &zero, sizeof(zero)) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+  }
+  if (raw_code != nullptr) *raw_code = v;
+  return v == 0 ? ATTN_OK : ATTN_ERR_TIMEOUT;
+}
+
+}  // extern "C"

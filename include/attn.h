@@ -1,0 +1,132 @@
+/*
+ * exact_tiled_attention_38_b200: exact scaled-dot-product attention for B200
+ * (sm_100a), as a C ABI.
+ *
+ * What is computed (every entry point): for each batch b, query head h and
+ * query row i,
+ *     s_ij  = scale * sum_c q[b,h,i,c] * k[b,g,j,c],   g = h / (Hq / Hkv)
+ *     s_ij  = -inf where key j is masked (causal: j > i + Nk - Nq)
+ *     o[b,h,i,:] = sum_j softmax_j(s_i.) * v[b,g,j,:]
+ *     lse[b,h,i] = ln sum_j exp(s_ij)
+ * This is exact attention (not an approximation): the aikaboom page
+ * "11.4d FlashAttention" lists the tiled method's result as the same
+ * mathematical result as standard attention (comparison table), and the
+ * zimaspace page "How Does Flash Attention Reduce Memory Traffic During Local
+ * Inference?" says the tiled algorithm still produces exact attention. It is
+ * computed tile by tile with a running (online) softmax, so the score matrix
+ * never reaches device memory (aikaboom page, sections "Tiling" and "Online
+ * Softmax"; zimaspace page, "Online Softmax Avoids Storing the Full Score
+ * Matrix" and "Kernel Fusion Keeps More of the Attention Chain in One
+ * Execution Path"). GQA grouping follows the sicorps page's last paragraph
+ * (n < n_head key/value heads, each shared by a group of query heads; MQA is
+ * Hkv = 1).
+ *
+ * Conventions shared by all entry points:
+ *   - All pointers are DEVICE pointers owned by the caller. The library never
+ *     frees or retains them. q, k, v, o, kcache, vcache must be 16-byte
+ *     aligned; lse and seqlens 4-byte aligned. Tensors are contiguous.
+ *   - Element type: attn_fwd / attn_decode take bfloat16 q, k, v and write
+ *     bfloat16 o; the _f16 twins take and write IEEE fp16. lse is float32.
+ *     Products accumulate in fp32; softmax statistics are fp32.
+ *   - scale must be finite and > 0 (the usual value is 1/sqrt(d)).
+ *   - lse may be NULL: the log-sum-exp is then not written.
+ *   - Work is enqueued on `stream` (NULL = legacy default stream); calls return
+ *     without synchronising. Errors detected on the host return a negative
+ *     code before anything is enqueued.
+ *   - A row with no visible key (causal with Nq > Nk, or an empty decode
+ *     sequence) gets o = 0 and lse = -inf.
+ *   - Every wait inside a kernel is bounded (about 2 s). If one gives up, the
+ *     kernel ends early, its outputs are undefined, and
+ *     attn_get_device_status() reports ATTN_ERR_TIMEOUT. No kernel traps.
+ */
+#ifndef EXACT_TILED_ATTENTION_ATTN_H
+#define EXACT_TILED_ATTENTION_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; declared here so that callers need no
+   CUDA header. */
+typedef struct CUstream_st* attn_stream_t;
+
+enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID = -1,     /* null pointer, bad size, misaligned, Hq % Hkv != 0, bad scale */
+  ATTN_ERR_UNSUPPORTED = -2, /* d not in {64, 128}, or the device is not sm_100 */
+  ATTN_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
+  ATTN_ERR_TIMEOUT = -4      /* a device-side wait gave up (see attn_get_device_status) */
+};
+
+/*
+ * Prefill: many query tokens against keys/values of the same sequence
+ * (aikaboom page, "The Core Problem" and "Tiling"; first page: prefill
+ * processes n tokens, so the cost is quadratic).
+ *   q   [B, Hq,  Nq, d]  bf16      k, v [B, Hkv, Nk, d] bf16
+ *   o   [B, Hq,  Nq, d]  bf16      lse  [B, Hq, Nq] float32 (or NULL)
+ *   causal != 0: bottom-right aligned mask, query i sees keys j <= i + Nk - Nq
+ *                (equal to the usual lower-triangular mask when Nq == Nk).
+ * Sizes: B >= 0, Nq >= 0, Nk >= 0 (B == 0 or Nq == 0: nothing to do;
+ * Nk == 0: every row is empty), Hq >= 1, Hkv >= 1, Hq % Hkv == 0,
+ * d in {64, 128}, Nq <= 16,776,960.
+ * Allocates no device memory.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, float scale, int causal, attn_stream_t stream);
+
+/* attn_fwd with IEEE fp16 q, k, v and o. */
+int attn_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                 int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                 attn_stream_t stream);
+
+/*
+ * Decode: one new query token per sequence over a ragged KV cache (first
+ * page: generating a token re-reads the whole KV cache plus the new entry, a
+ * cost linear in the cache length; zimaspace page, "Reduced IO Is Not the Same
+ * as Eliminating KV Cache").
+ *   q       [B, Hq, d]  bf16
+ *   kcache, vcache: packed per sequence. Sequence b starts at token offset
+ *           off_b = sum_{j<b} seqlens[j] and is laid out [Hkv][seqlens[b]][d],
+ *           i.e. element (b, g, t, c) is at ((off_b * Hkv + g * L_b + t) * d + c).
+ *           The new token's key/value must already be appended.
+ *           kcache and vcache must be non-NULL even if every sequence is empty.
+ *   seqlens [B] int32, DEVICE memory, read only on the device (negative
+ *           values count as 0; 0 gives o = 0, lse = -inf).
+ *   o       [B, Hq, d]  bf16       lse [B, Hq] float32 (or NULL)
+ * Sizes: B >= 0 (0: nothing to do), Hq >= 1, Hkv >= 1, Hq % Hkv == 0,
+ * d in {64, 128}.
+ * Allocates a split-KV scratch of nsplit * B * Hq * (d + 1) * 4 bytes with
+ * cudaMallocAsync on `stream` and frees it with cudaFreeAsync on the same
+ * stream (stream-ordered; nothing outlives the call's work).
+ */
+int attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
+                attn_stream_t stream);
+
+/* attn_decode with IEEE fp16 q, kcache, vcache and o. */
+int attn_decode_f16(const void* q, const void* kcache, const void* vcache,
+                    const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv, int d,
+                    float scale, attn_stream_t stream);
+
+/* Number of KV splits attn_decode uses for these sizes on the current device
+   (>= 1), or a negative error code. */
+int attn_decode_num_splits(int B, int Hq, int Hkv, int d);
+
+/* Human-readable text for a return code. Never NULL. */
+const char* attn_strerror(int code);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device status
+ * word on the current device. Returns ATTN_OK, ATTN_ERR_TIMEOUT (a device
+ * wait gave up; *raw_code, if not NULL, receives the site code) or
+ * ATTN_ERR_CUDA.
+ */
+int attn_get_device_status(attn_stream_t stream, unsigned int* raw_code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_TILED_ATTENTION_ATTN_H */

@@ -111,12 +111,14 @@ def _head_ref(qh: np.ndarray, kh: np.ndarray, vh: np.ndarray, scale: float,
     return o, lse
 
 
-def attention_ref(q, k, v, scale: float, causal: bool, rows=None):
+def attention_ref(q, k, v, scale: float, causal: bool, rows=None, nq=None):
     """Exact attention in fp64.
 
     q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] (any float dtype; converted exactly).
     rows: None (every query row), a 1-D array of row indices used for every
     head, or an integer array [B, Hq, R] of per-head rows.
+    nq: when given, q holds only the query rows listed in the 1-D ``rows`` (in
+    that order) and nq is the full query length the causal mask refers to.
     Returns (O [B, Hq, R, d], LSE [B, Hq, R]) in float64; R = Nq when rows is None.
     """
     q = _f64(q)
@@ -129,6 +131,18 @@ def attention_ref(q, k, v, scale: float, causal: bool, rows=None):
     if Hq % Hkv != 0:
         raise ValueError("Hq must be a multiple of Hkv")
     group = Hq // Hkv
+    if nq is not None:
+        rows_arr = np.asarray(rows, dtype=np.int64)
+        if rows_arr.ndim != 1 or rows_arr.size != Nq:
+            raise ValueError("with nq, rows must list the rows q holds")
+        out = np.zeros((B, Hq, Nq, d))
+        lse = np.zeros((B, Hq, Nq))
+        for b in range(B):
+            for h in range(Hq):
+                g = h // group
+                out[b, h], lse[b, h] = _head_ref(q[b, h], k[b, g], v[b, g], scale, causal,
+                                                 nq, rows_arr)
+        return out, lse
     if rows is None:
         rows_arr = np.broadcast_to(np.arange(Nq), (B, Hq, Nq))
     else:
@@ -147,17 +161,33 @@ def attention_ref(q, k, v, scale: float, causal: bool, rows=None):
     return out, lse
 
 
-def unpack_decode_cache(cache, seqlens, Hkv: int, d: int):
-    """Split a packed decode cache into per-sequence [Hkv, L_b, d] fp64 arrays."""
-    flat = _f64(cache).reshape(-1)
+def _sequence_ranges(seqlens, Hkv: int, d: int):
+    """(start, L) element ranges of each sequence's block in a packed cache."""
     lens = [max(0, int(x)) for x in _f64(seqlens).reshape(-1)]
-    parts = []
+    out = []
     off = 0
     for L in lens:
-        n = L * Hkv * d
-        parts.append(flat[off:off + n].reshape(Hkv, L, d))
-        off += n
-    return parts
+        out.append((off, L))
+        off += L * Hkv * d
+    return out
+
+
+def _flat(cache):
+    try:
+        import torch
+
+        if isinstance(cache, torch.Tensor):
+            return cache.detach().reshape(-1)
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(cache).reshape(-1)
+
+
+def unpack_decode_cache(cache, seqlens, Hkv: int, d: int):
+    """Split a packed decode cache into per-sequence [Hkv, L_b, d] fp64 arrays."""
+    flat = _flat(cache)
+    return [_f64(flat[o:o + L * Hkv * d]).reshape(Hkv, L, d)
+            for o, L in _sequence_ranges(seqlens, Hkv, d)]
 
 
 def decode_ref(q, kcache, vcache, seqlens, scale: float, Hkv: int):
@@ -167,20 +197,21 @@ def decode_ref(q, kcache, vcache, seqlens, scale: float, Hkv: int):
     seqlens: [B] ints. Returns (O [B, Hq, d], LSE [B, Hq]).
     Each new token reads the whole cache of its sequence (the "token generation"
     case on the first page: linear in the number of cached entries).
+    Sequences are converted to fp64 one at a time, so large caches fit in memory.
     """
     q = _f64(q)
     B, Hq, d = q.shape
-    ks = unpack_decode_cache(kcache, seqlens, Hkv, d)
-    vs = unpack_decode_cache(vcache, seqlens, Hkv, d)
+    kf = _flat(kcache)
+    vf = _flat(vcache)
     out = np.zeros((B, Hq, d))
     lse = np.zeros((B, Hq))
-    for b in range(B):
-        L = ks[b].shape[1]
+    for b, (o0, L) in enumerate(_sequence_ranges(seqlens, Hkv, d)):
         if L == 0:
             lse[b] = -np.inf
             continue
-        o, l = attention_ref(q[b][None, :, None, :], ks[b][None], vs[b][None], scale,
-                             causal=False)
+        kb = _f64(kf[o0:o0 + L * Hkv * d]).reshape(1, Hkv, L, d)
+        vb = _f64(vf[o0:o0 + L * Hkv * d]).reshape(1, Hkv, L, d)
+        o, l = attention_ref(q[b][None, :, None, :], kb, vb, scale, causal=False)
         out[b] = o[0, :, 0]
         lse[b] = l[0, :, 0]
     return out, lse

@@ -1,0 +1,119 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+The library must load, export every function declared in include/attn.h with
+the signature the binding declares, and reject bad arguments on the host
+before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_tiled_attention_38_b200 as eta
+from exact_tiled_attention_38_b200 import build as eta_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def clib():
+    eta_build.build()
+    return eta.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(attn_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("attn_fwd", "attn_decode", "attn_fwd_f16", "attn_decode_f16", "attn_strerror",
+              "attn_get_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(clib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(clib, n), f"{n} not exported"
+    assert set(names) == set(eta.SIGNATURES), "binding and header disagree"
+
+
+def test_argument_counts_match_header():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    for name, (_, args) in eta.SIGNATURES.items():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", text)
+        assert m, name
+        params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        assert len(params) == len(args), name
+
+
+def test_strerror_covers_codes(clib):
+    for code in (eta.ATTN_OK, eta.ATTN_ERR_INVALID, eta.ATTN_ERR_UNSUPPORTED, eta.ATTN_ERR_CUDA,
+                 eta.ATTN_ERR_TIMEOUT, 12345):
+        s = clib.attn_strerror(code)
+        assert s and len(s) > 1
+
+
+# Calls that the host rejects (or finds empty) before touching CUDA.
+FAKE = ctypes.c_void_p(0x10000)
+
+
+def fwd(clib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=4, Hkv=2, Nq=8, Nk=8, d=128,
+             scale=0.1, causal=1)
+    a.update(kw)
+    return clib.attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                         a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"], None)
+
+
+def test_fwd_host_validation(clib):
+    assert fwd(clib, Hq=3) == eta.ATTN_ERR_INVALID
+    assert fwd(clib, Hkv=0) == eta.ATTN_ERR_INVALID
+    assert fwd(clib, B=-1) == eta.ATTN_ERR_INVALID
+    assert fwd(clib, Nq=-5) == eta.ATTN_ERR_INVALID
+    assert fwd(clib, scale=0.0) == eta.ATTN_ERR_INVALID
+    assert fwd(clib, scale=float("inf")) == eta.ATTN_ERR_INVALID
+    assert fwd(clib, d=96) == eta.ATTN_ERR_UNSUPPORTED
+    assert fwd(clib, d=256) == eta.ATTN_ERR_UNSUPPORTED
+    assert fwd(clib, o=None) == eta.ATTN_ERR_INVALID
+    assert fwd(clib, q=ctypes.c_void_p(0x10008)) == eta.ATTN_ERR_INVALID
+    assert fwd(clib, lse=ctypes.c_void_p(0x10002)) == eta.ATTN_ERR_INVALID
+    assert fwd(clib, Nq=65535 * 256 + 1) == eta.ATTN_ERR_INVALID
+    # empty problems are a no-op
+    assert fwd(clib, B=0) == eta.ATTN_OK
+    assert fwd(clib, Nq=0) == eta.ATTN_OK
+    assert clib.attn_fwd_f16(FAKE, FAKE, FAKE, FAKE, None, 0, 1, 1, 4, 4, 64, 0.1, 0,
+                             None) == eta.ATTN_OK
+
+
+def dec(clib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, s=FAKE, o=FAKE, lse=None, B=2, Hq=8, Hkv=2, d=128,
+             scale=0.1)
+    a.update(kw)
+    return clib.attn_decode(a["q"], a["k"], a["v"], a["s"], a["o"], a["lse"], a["B"], a["Hq"],
+                            a["Hkv"], a["d"], a["scale"], None)
+
+
+def test_decode_host_validation(clib):
+    assert dec(clib, Hq=6, Hkv=4) == eta.ATTN_ERR_INVALID
+    assert dec(clib, scale=-0.5) == eta.ATTN_ERR_INVALID
+    assert dec(clib, d=80) == eta.ATTN_ERR_UNSUPPORTED
+    assert dec(clib, s=None) == eta.ATTN_ERR_INVALID
+    assert dec(clib, s=ctypes.c_void_p(0x10002)) == eta.ATTN_ERR_INVALID
+    assert dec(clib, k=ctypes.c_void_p(0x10004)) == eta.ATTN_ERR_INVALID
+    assert dec(clib, B=0) == eta.ATTN_OK
+    assert clib.attn_decode_num_splits(2, 6, 4, 128) == eta.ATTN_ERR_INVALID
+    assert clib.attn_decode_num_splits(2, 8, 2, 96) == eta.ATTN_ERR_UNSUPPORTED
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(eta, "_lib", None)
+    with pytest.raises(RuntimeError):
+        eta.load_library(str(tmp_path / "missing.so"))

@@ -396,3 +396,13 @@ def test_pins_catch_planted_mistakes(monkeypatch):
                 m.setattr(oracle, "attention_ref", fn)
             assert not _all_pins_pass(), f"planted mistake {fn.__name__} went unnoticed"
     assert oracle_mod._visible is good_visible and oracle_mod.scores is good_scores
+
+
+def test_subset_query_rows_with_full_length():
+    q = _rand((1, 2, 30, 8), 96)
+    k = _rand((1, 1, 30, 8), 97)
+    v = _rand((1, 1, 30, 8), 98)
+    rows = np.array([0, 5, 17, 29])
+    o, lse = oracle.attention_ref(q, k, v, 0.4, True, rows=rows)
+    o2, lse2 = oracle.attention_ref(q[:, :, rows], k, v, 0.4, True, rows=rows, nq=30)
+    assert np.abs(o - o2).max() == 0.0 and np.abs(lse - lse2).max() == 0.0
