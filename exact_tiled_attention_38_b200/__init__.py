@@ -21,6 +21,7 @@ ATTN_ERR_INVALID = -1
 ATTN_ERR_UNSUPPORTED = -2
 ATTN_ERR_CUDA = -3
 ATTN_ERR_TIMEOUT = -4
+ATTN_ERR_SCRATCH = -5
 
 # name -> (restype, argtypes); mirrors include/attn.h
 _P = ctypes.c_void_p
@@ -31,6 +32,7 @@ SIGNATURES = {
     "attn_fwd_f16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "attn_decode_f16": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
+    "attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "attn_decode_num_splits": (_I, [_I, _I, _I, _I]),
     "attn_strerror": (ctypes.c_char_p, [_I]),
     "attn_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
@@ -182,6 +184,21 @@ def attn_decode_f16(q, kcache, vcache, seqlens, Hkv: int, o=None, lse=None,
 
     return _decode("attn_decode_f16", torch.float16, q, kcache, vcache, seqlens, Hkv, o, lse,
                    scale, stream, want_lse)
+
+
+def attn_decode_noalloc(q, kcache, vcache, seqlens, Hkv: int, o=None, lse=None,
+                        scale: Optional[float] = None, stream=None, want_lse: bool = True):
+    """bf16 decode whose scratch is the library's fixed device array.
+
+    For callers that cannot allocate device memory where decode runs. The
+    library allocates nothing here; pass preallocated ``o`` / ``lse`` to keep
+    this wrapper from allocating them either. Calls that may overlap on the GPU
+    share the scratch and must be ordered (one stream, or events).
+    """
+    import torch
+
+    return _decode("attn_decode_noalloc", torch.bfloat16, q, kcache, vcache, seqlens, Hkv, o,
+                   lse, scale, stream, want_lse)
 
 
 def attn_decode_num_splits(B: int, Hq: int, Hkv: int, d: int) -> int:

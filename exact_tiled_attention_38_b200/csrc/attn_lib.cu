@@ -312,6 +312,9 @@ const char* attn_strerror(int code) {
       return "CUDA runtime error";
     case ATTN_ERR_TIMEOUT:
       return "a device-side wait gave up; outputs of that launch are undefined";
+    case ATTN_ERR_SCRATCH:
+      return "B * Hq * (d + 1) exceeds the fixed scratch of attn_decode_noalloc "
+             "(2,097,152 floats)";
     default:
       return "unknown error code";
   }
@@ -332,3 +335,101 @@ int attn_get_device_status(attn_stream_t stream, unsigned int* raw_code) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without any allocation.
+//
+// attn_decode takes its split-KV scratch from cudaMallocAsync. Some callers
+// cannot allocate device memory at the point where they run attention: a
+// serving engine that hands nearly all of HBM to its own KV-cache pool at
+// start-up (so an extra allocation can fail, or fragment that pool), code on a
+// latency-critical path where an allocator call may take a lock or synchronise,
+// and runtimes that fix their whole memory plan before the first request. For
+// them, attn_decode_noalloc runs the same two decode kernels with the scratch
+// taken from a fixed array in this library's device memory instead.
+namespace eta {
+namespace api {
+
+// Capacity of the fixed scratch, in floats (8 MiB). Every GPU that loads the
+// library holds this much device memory until the process exits.
+constexpr size_t kNoAllocScratchFloats = size_t(2) << 20;
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+// On the host, g_noalloc_scratch names a host-side stand-in, not device
+// memory: a kernel handed that name would fault or, where the GPU can reach
+// host memory, silently use the wrong memory. The device address is looked up
+// here, once per device, with that device current.
+int noalloc_scratch(float** out) {
+  static std::mutex mu;
+  static float* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return ATTN_ERR_CUDA;
+    addr[dev] = static_cast<float*>(p);
+  }
+  *out = addr[dev];
+  return ATTN_OK;
+}
+
+template <typename T>
+int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int32_t* seqlens,
+                       void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
+                       cudaStream_t st) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale)) return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq > 0x7fffffffLL / 4) return ATTN_ERR_INVALID;
+  if (B == 0) return ATTN_OK;
+  if (q == nullptr || kc == nullptr || vc == nullptr || seqlens == nullptr || o == nullptr ||
+      !aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(o, 16) ||
+      !aligned(seqlens, 4) || (lse != nullptr && !aligned(lse, 4)))
+    return ATTN_ERR_INVALID;
+  // One split needs B * Hq * (d + 1) floats; fewer splits are used when the
+  // usual count does not fit, and sizes where even one does not fit are refused.
+  const size_t rows = static_cast<size_t>(B) * Hq;
+  const size_t per_split = rows * (d + 1);
+  if (per_split > kNoAllocScratchFloats) return ATTN_ERR_SCRATCH;
+  DeviceInfo info;
+  if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
+  float* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != ATTN_OK) return ATTN_ERR_CUDA;
+
+  decode::DParams p;
+  p.q = q;
+  p.kc = kc;
+  p.vc = vc;
+  p.seqlens = seqlens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  const int GP = p.G <= 4 ? 4 : 8;
+  p.nchunk = (p.G + GP - 1) / GP;
+  const size_t fit = kNoAllocScratchFloats / per_split;
+  const int want = decode_splits(B, Hq, Hkv, d, info.sm_count);
+  p.nsplit = static_cast<int>(fit < static_cast<size_t>(want) ? fit : want);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_ns = kDefaultWaitNs;
+  // Every partial slot is written by the split pass before the combine reads
+  // it, so nothing in the scratch has to start at zero.
+  p.part_o = scratch;
+  p.part_lse = scratch + static_cast<size_t>(p.nsplit) * rows * d;
+  return d == 128 ? decode_launch_all<128, T>(p, o, lse, st)
+                  : decode_launch_all<64, T>(p, o, lse, st);
+}
+
+}  // namespace api
+}  // namespace eta
+
+extern "C" int attn_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                                   const int32_t* seqlens, void* o, float* lse, int B, int Hq,
+                                   int Hkv, int d, float scale, attn_stream_t stream) {
+  return eta::api::decode_run_noalloc<__nv_bfloat16>(q, kcache, vcache, seqlens, o, lse, B, Hq,
+                                                     Hkv, d, scale,
+                                                     reinterpret_cast<cudaStream_t>(stream));
+}

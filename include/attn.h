@@ -57,7 +57,8 @@ enum attn_status {
   ATTN_ERR_INVALID = -1,     /* null pointer, bad size, misaligned, Hq % Hkv != 0, bad scale */
   ATTN_ERR_UNSUPPORTED = -2, /* d not in {64, 128}, or the device is not sm_100 */
   ATTN_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
-  ATTN_ERR_TIMEOUT = -4      /* a device-side wait gave up (see attn_get_device_status) */
+  ATTN_ERR_TIMEOUT = -4,     /* a device-side wait gave up (see attn_get_device_status) */
+  ATTN_ERR_SCRATCH = -5      /* attn_decode_noalloc: sizes exceed its fixed scratch */
 };
 
 /*
@@ -109,6 +110,32 @@ int attn_decode(const void* q, const void* kcache, const void* vcache, const int
 int attn_decode_f16(const void* q, const void* kcache, const void* vcache,
                     const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv, int d,
                     float scale, attn_stream_t stream);
+
+/*
+ * attn_decode that allocates nothing. The pages have no counterpart for this
+ * entry point; it exists for callers that cannot allocate device memory where
+ * they run decode: an engine that gives nearly all of HBM to its own KV-cache
+ * pool at start-up, a latency-critical path where an allocator call may lock
+ * or synchronise, or a runtime whose memory plan is fixed before serving.
+ * Same arguments, layout and results as attn_decode (bf16), except:
+ *   - The split-KV scratch is a fixed array of 2,097,152 floats (8 MiB) in
+ *     this library's device memory, held by every GPU that loads the library
+ *     until the process exits. It calls no cudaMalloc/cudaFree and no
+ *     allocating library routine.
+ *   - One split needs B * Hq * (d + 1) floats. When the usual split count does
+ *     not fit, fewer splits are used (results then agree with attn_decode to
+ *     rounding); when even one split does not fit, the call returns
+ *     ATTN_ERR_SCRATCH and enqueues nothing.
+ *   - The first call on a device looks up the array's device address (a
+ *     runtime call); make that first call before any stream capture.
+ *   - Every call on a device uses the same array, which keeps the previous
+ *     call's contents (nothing in it needs to start at zero). Calls that can
+ *     overlap on the GPU (different streams without ordering between them)
+ *     race on it and give wrong results; order them on one stream or by events.
+ */
+int attn_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                        const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                        int d, float scale, attn_stream_t stream);
 
 /* Number of KV splits attn_decode uses for these sizes on the current device
    (>= 1), or a negative error code. */

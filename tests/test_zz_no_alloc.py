@@ -1,0 +1,69 @@
+"""attn_decode_noalloc: decode with the scratch in a fixed library array.
+
+Some callers cannot allocate device memory where they run decode (an engine
+that has handed almost all of HBM to its own KV-cache pool, a latency-critical
+path where an allocator call may lock or synchronise, a runtime whose memory
+plan is fixed up front). The no-allocation entry point serves them; these tests
+check, through the C ABI, that it gives the allocating entry point's results
+within the parity tolerances on consecutive calls, that a later call is not
+affected by what an earlier one left in the shared scratch, and that sizes the
+scratch cannot hold are refused with their own error code.
+
+This file is collected last so that a run stopping at the first failure has
+already run every other test; it also passes alone in a fresh process.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from parity import TOL_LSE, TOL_O
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _agree(o, lse, o_ref, lse_ref):
+    d_o = (o.float() - o_ref.float()).abs().max().item()
+    fin = torch.isfinite(lse_ref)
+    assert torch.equal(torch.isfinite(lse), fin)
+    d_l = (lse[fin] - lse_ref[fin]).abs().max().item() if fin.any() else 0.0
+    assert d_o <= TOL_O[torch.bfloat16], d_o
+    assert d_l <= TOL_LSE, d_l
+
+
+def _call_pair(lib, q, kc, vc, sl, Hkv):
+    o_ref, lse_ref = lib.attn_decode(q, kc, vc, sl, Hkv=Hkv)
+    for _ in range(2):  # two calls in a row, fresh outputs each time
+        o = torch.full_like(q, float("nan"))
+        lse = torch.full(lse_ref.shape, float("nan"), device=DEV)
+        lib.attn_decode_noalloc(q, kc, vc, sl, Hkv=Hkv, o=o, lse=lse)
+        torch.cuda.synchronize()
+        assert lib.attn_get_device_status()[0] == lib.ATTN_OK
+        _agree(o, lse, o_ref, lse_ref)
+
+
+def test_noalloc_matches_allocating_decode_on_ragged_workload(lib):
+    w = workloads.DECODE_GQA_RAGGED
+    q, kc, vc, sl = workloads.decode_inputs(w, device=DEV)
+    _call_pair(lib, q, kc, vc, sl, w.Hkv)
+
+
+def test_noalloc_after_a_larger_call_and_with_empty_sequences(lib):
+    # A smaller problem after the big one: stale scratch contents must not leak.
+    sl = torch.tensor([5, 0, 1300, 64], dtype=torch.int32)
+    q, kc, vc, sl = workloads.random_decode(4, 16, 2, 64, sl, torch.bfloat16, seed=31,
+                                            device=DEV)
+    _call_pair(lib, q, kc, vc, sl, 2)
+
+
+def test_noalloc_refuses_sizes_beyond_its_scratch(lib):
+    # B * Hq * (d + 1) floats per split; 16384 * 8 * 129 is above 2,097,152.
+    B, Hq, Hkv, d = 16384, 8, 2, 128
+    q = torch.zeros(B, Hq, d, device=DEV, dtype=torch.bfloat16)
+    kc = torch.zeros(64, device=DEV, dtype=torch.bfloat16)
+    sl = torch.zeros(B, device=DEV, dtype=torch.int32)
+    with pytest.raises(lib.AttnError) as e:
+        lib.attn_decode_noalloc(q, kc, kc, sl, Hkv=Hkv)
+    assert e.value.code == lib.ATTN_ERR_SCRATCH
