@@ -24,7 +24,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -139,34 +138,66 @@ def aggregate_throughput(units_per_rank: float, world: int, max_ms: float) -> fl
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples nvidia-smi SM clocks and throttle reasons while the timed loop runs."""
+    """Samples SM clocks and clock-event (throttle) reasons through NVML, read
+    only, every 20 ms while the timed loop runs. The GPU is matched by PCI bus id
+    so that NVML and CUDA indices need not agree."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {  # NVML clocks-event reason bits that reject or annotate a run
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4,
+    }
 
-    def __init__(self, index: int):
-        self.index = index
-        self.rows = []
+    def __init__(self, cuda_index: int, period_s: float = 0.02):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.sm = []
+        self.max_sm = None
+        self.reasons = set()
+        self.error = None
         self._stop = threading.Event()
         self._t = None
+        self._h = None
+        self._nvml = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+
+        pynvml.nvmlInit()
+        self._nvml = pynvml
+        props = torch.cuda.get_device_properties(self.cuda_index)
+        bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id,
+                                    props.pci_device_id)
+        try:
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def _run(self):
-        while not self._stop.is_set():
+        nv = self._nvml
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while True:
             try:
-                out = subprocess.run(
-                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                     "--format=csv,noheader,nounits"], capture_output=True, text=True,
-                    timeout=5).stdout.strip()
-                if out:
-                    self.rows.append([x.strip() for x in out.split(",")])
-            except Exception:
+                self.sm.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = get_reasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if bits & bit:
+                        self.reasons.add(name)
+            except Exception as e:  # pragma: no cover
+                self.error = str(e)
                 return
-            self._stop.wait(0.1)
+            if self._stop.wait(self.period):
+                return
 
     def __enter__(self):
-        self._t = threading.Thread(target=self._run, daemon=True)
-        self._t.start()
+        try:
+            self._h = self._handle()
+            self.max_sm = self._nvml.nvmlDeviceGetMaxClockInfo(self._h, self._nvml.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception as e:
+            self.error = str(e)
         return self
 
     def __exit__(self, *a):
@@ -175,16 +206,12 @@ class ClockSampler:
             self._t.join(timeout=10)
 
     def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4)
-                          if len(r) > 5 + i and r[5 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.rows)}
+        out = {"sm_mhz": statistics.median(self.sm) if self.sm else None,
+               "sm_max_mhz": self.max_sm, "reasons": sorted(self.reasons),
+               "samples": len(self.sm), "source": "nvml"}
+        if self.error:
+            out["error"] = self.error
+        return out
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -466,19 +493,53 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+def run_profile(args, local):
+    """Launch one phase of the step `warmup + steps` times with no timing or
+    output: the target of an ncu capture (a small, self-contained command)."""
+    import torch
+
+    import exact_tiled_attention_38_b200 as eta
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    eta.load_library()
+    if args.profile in ("prefill", "prefill_32k"):
+        w = PREFILL if args.profile == "prefill" else workloads.PREFILL_GQA_32K
+        q, k, v = workloads.prefill_inputs(w, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty(w.B, w.Hq, w.Nq, device=dev, dtype=torch.float32)
+        for _ in range(args.warmup + args.steps):
+            eta.attn_fwd(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal)
+    else:
+        dq, dkc, dvc, dsl = workloads.decode_inputs(DECODE, device=dev)
+        do = torch.empty_like(dq)
+        dlse = torch.empty(DECODE.B, DECODE.Hq, device=dev, dtype=torch.float32)
+        for _ in range(args.warmup + args.steps):
+            eta.attn_decode(dq, dkc, dvc, dsl, DECODE.Hkv, o=do, lse=dlse, scale=DECODE.scale)
+    torch.cuda.synchronize()
+    code, raw = eta.attn_get_device_status()
+    if code != eta.ATTN_OK:
+        raise RuntimeError(f"device status {code} ({raw:#x})")
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1500)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=("prefill", "prefill_32k", "decode"), default=None,
+                    help="only launch this phase (an ncu target); prints nothing")
     args = ap.parse_args(argv)
-    if args.warmup < 3:
+    if args.warmup < 3 and not args.profile:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.profile:
+        return run_profile(args, local)
     return run_ours(args, world, rank, local)
 
 

@@ -106,10 +106,16 @@ int launch_fill_empty(void* o, float* lse, long long rows, int D, cudaStream_t s
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Prefill kernel knob: POLY8 of every 8 score columns take 2^x from the FMA
+// polynomial instead of the special-function unit.
+#ifndef ETA_PREFILL_POLY8
+#define ETA_PREFILL_POLY8 0
+#endif
+
 template <int D, typename T, bool CAUSAL>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const prefill::Params& p, int B, cudaStream_t st) {
-  auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL>;
+                   const prefill::Params& p, int grid, cudaStream_t st) {
+  auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, ETA_PREFILL_POLY8, false>;
   constexpr int smem = prefill::Cfg<D>::kSmemBytes;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -117,7 +123,6 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>(B) * p.Hq, static_cast<unsigned>(p.n_pairs));
   kern<<<grid, prefill::kThreads, smem, st>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -159,14 +164,19 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   p.group = Hq / Hkv;
   p.n_pairs = (Nq + prefill::NQT * prefill::BM - 1) / (prefill::NQT * prefill::BM);
   p.off = Nk - Nq;
+  p.BH = B * Hq;
+  const long long total = static_cast<long long>(p.BH) * p.n_pairs;
+  if (total > 0x7fffffffLL) return ATTN_ERR_INVALID;
+  p.total = static_cast<int>(total);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = wait_ns;
   p.debug_flags = debug_flags;
+  const int grid = static_cast<int>(total < info.sm_count ? total : info.sm_count);
   if (d == 128)
-    return causal ? launch_prefill<128, T, true>(tq, tk, tv, p, B, st)
-                  : launch_prefill<128, T, false>(tq, tk, tv, p, B, st);
-  return causal ? launch_prefill<64, T, true>(tq, tk, tv, p, B, st)
-                : launch_prefill<64, T, false>(tq, tk, tv, p, B, st);
+    return causal ? launch_prefill<128, T, true>(tq, tk, tv, p, grid, st)
+                  : launch_prefill<128, T, false>(tq, tk, tv, p, grid, st);
+  return causal ? launch_prefill<64, T, true>(tq, tk, tv, p, grid, st)
+                : launch_prefill<64, T, false>(tq, tk, tv, p, grid, st);
 }
 
 // Split-KV count: enough CTAs for about eight waves of resident split CTAs.

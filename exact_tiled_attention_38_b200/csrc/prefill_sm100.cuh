@@ -9,13 +9,16 @@
 // max and row sum are carried from key tile to key tile, and scaling, masking,
 // normalisation and the value product all stay inside one kernel.
 //
-// One CTA owns two 128-row query tiles of one (batch, query head) and streams
-// the key/value tiles of that head's KV head (GQA: kv head = h / (Hq / Hkv)).
+// Work items are pairs of 128-row query tiles of one (batch, query head). The
+// grid is persistent (one CTA per SM); CTA c takes items c, 2G-1-c, 2G+c, ...
+// (G = grid size) from a list ordered heaviest first for causal masks, which
+// balances the triangular work. Each item streams the key/value tiles of its
+// KV head (GQA: kv head = h / (Hq / Hkv)).
 // Warp roles (320 threads):
 //   warps 0-3  softmax for query tile 0 (one thread per query row)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    tensor-memory owner and the single thread that issues tcgen05.mma
-//   warp  9    TMA producer: Q once, then K_j and V_j through a ring of stages
+//   warp  9    TMA producer: Q tiles, then K_j and V_j through a ring of stages
 // Tensor memory (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256),
 // O_0 [256, 256+D), O_1 [256+D, 256+2D); the bf16/fp16 probabilities P_t
 // overwrite columns [64,128) of S_t once the softmax has read S_t. The MMA
@@ -23,7 +26,8 @@
 // for t = 0, 1, so while one softmax group works on its tile the tensor core
 // runs the other group's products. tcgen05.mma operations issued by one thread
 // execute in issue order, which is what lets S_t(j) reuse the columns that
-// P_t(j-1) occupied.
+// P_t(j-1) occupied. The next item's Q loads and first S products overlap the
+// current item's epilogue.
 //
 // Online softmax per row (fp32, log2 domain, c = scale * log2 e):
 //   m' = max over the tile of s * c; if m' > m + 8 the row's running max moves
@@ -31,6 +35,13 @@
 //   kept (exact: O and l share the same reference, p <= 2^8).
 //   p = 2^(s*c - m), l += sum p (unrounded), P = round(p) -> tensor memory.
 // Epilogue: O / l rounded to the input type; LSE = ln 2 * (m + log2 l).
+//
+// Two optional refinements (template knobs):
+//   PINGPONG  the two softmax groups take turns (an mbarrier token) for their
+//             exponential phase, so the special-function unit serves one group
+//             while the tensor core serves the other;
+//   POLY8     of every 8 score columns, POLY8 get 2^x from a polynomial on the
+//             FMA pipe (ex2_poly) instead of the special-function unit.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -62,6 +73,8 @@ enum : unsigned {
   kSiteSReady = 5,
   kSiteODone = 6,
   kSiteDrain = 7,
+  kSiteQEmpty = 8,
+  kSiteTurn = 9,
 };
 
 template <int D>
@@ -74,7 +87,9 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = NQT * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kStages + 3 * NQT + 1;
+  // kv_full[S], kv_empty[S], then per tile: q_full, q_empty, s_ready, p_ready,
+  // o_done, turn; then drain.
+  static constexpr int kNumBars = 2 * kStages + 6 * NQT + 1;
   static constexpr int kCtlOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kCtlOff + 64 + 1024;  // + runtime 1024-byte alignment
   static constexpr uint32_t kOCol = 2 * BN;
@@ -90,6 +105,8 @@ struct Params {
   int group;       // Hq / Hkv
   int n_pairs;     // ceil(Nq / 256)
   int off;         // Nk - Nq: query i sees keys j <= i + off when causal
+  int BH;          // B * Hq
+  int total;       // BH * n_pairs work items
   float scale_log2;
   uint64_t wait_ns;
   int debug_flags;  // bit 0: the producer issues no copies (exercises the wait limit)
@@ -123,7 +140,124 @@ struct Fmt<__half> {
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
-template <int D, typename T, bool CAUSAL>
+// 2^x on the FMA and integer pipes, for x <= 8.
+// Range reduction: n = round(x) (adding 1.5 * 2^23 leaves round(x) in the low
+// mantissa bits; exact for |x| < 2^22), f = x - n in [-1/2, 1/2], so
+// 2^x = 2^n * 2^f. 2^f is a degree-3 polynomial whose coefficients are the
+// minimax fit for relative error on [-1/2, 1/2], obtained with the Remez
+// exchange algorithm: max relative error 7.5e-5 (2^-13.7), below the rounding
+// of P to bf16 (2^-9) or fp16 (2^-11). 2^n is applied by adding n to the
+// exponent field.
+constexpr float kExp2C0 = 0.99992805719375610f;
+constexpr float kExp2C1 = 0.69326096773147583f;
+constexpr float kExp2C2 = 0.24261112511157990f;
+constexpr float kExp2C3 = 0.05517166852951050f;
+
+// Two values at once: the adds and the polynomial run as fp32-pair
+// instructions. Inputs are clamped to -126 first, so the exponent field never
+// underflows; callers use this only where no score is masked (2^-126 stands in
+// for anything smaller).
+__device__ __forceinline__ uint64_t ex2_poly2(float x0, float x1) {
+  const uint64_t x = f2_make(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t magic = f2_make(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t n = f2_add(t, f2_make(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_fma(n, f2_make(-1.0f, -1.0f), x);
+  uint64_t q = f2_fma(f2_make(kExp2C3, kExp2C3), f, f2_make(kExp2C2, kExp2C2));
+  q = f2_fma(q, f, f2_make(kExp2C1, kExp2C1));
+  q = f2_fma(q, f, f2_make(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2_split(q, q0, q1);
+  f2_split(t, t0, t1);
+  const float r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  const float r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+  return f2_make(r0, r1);
+}
+
+struct Item {
+  int bh;
+  int b;
+  int kvh;
+  int r0;  // first query row of tile 0 (tile 1 starts at r0 + BM)
+  int n0;  // key tiles for query tile 0
+  int n1;  // key tiles for query tile 1
+};
+
+// Snake order over the persistent grid: balances items sorted heaviest first.
+__device__ __forceinline__ int item_index(int round, int cta, int G) {
+  return round * G + ((round & 1) ? (G - 1 - cta) : cta);
+}
+
+template <bool CAUSAL>
+__device__ __forceinline__ int key_tiles(int r0, const Params& p, int nkv_all) {
+  if (r0 >= p.Nq) return 0;
+  if (!CAUSAL) return nkv_all;
+  const int last_row = min(r0 + BM - 1, p.Nq - 1);
+  const long long kmax = static_cast<long long>(last_row) + p.off;
+  if (kmax < 0) return 0;
+  const long long ntiles = kmax / BN + 1;
+  return static_cast<int>(ntiles < nkv_all ? ntiles : nkv_all);
+}
+
+template <bool CAUSAL>
+__device__ __forceinline__ Item decode_item(int idx, const Params& p, int nkv_all) {
+  Item it;
+  int pair;
+  if (CAUSAL) {  // heaviest (last) query tiles first, all heads of one level together
+    pair = p.n_pairs - 1 - idx / p.BH;
+    it.bh = idx - (idx / p.BH) * p.BH;
+  } else {  // consecutive items share a head, so concurrent CTAs share K/V in L2
+    it.bh = idx / p.n_pairs;
+    pair = idx - it.bh * p.n_pairs;
+  }
+  it.b = it.bh / p.Hq;
+  const int h = it.bh - it.b * p.Hq;
+  it.kvh = h / p.group;
+  it.r0 = pair * (NQT * BM);
+  it.n0 = key_tiles<CAUSAL>(it.r0, p, nkv_all);
+  it.n1 = key_tiles<CAUSAL>(it.r0 + BM, p, nkv_all);
+  return it;
+}
+
+// p = 2^(s * c - m) for one row of a score tile: writes P (rounded to T) to
+// tensor memory at tP, 32 columns at a time, and returns the fp32 sum of p.
+// POLY8 of every 8 columns use the polynomial exponential (only for tiles
+// without masked scores).
+template <typename T, int POLY8>
+__device__ __forceinline__ float exp_tile(const float (&s)[BN], float c, float m_use, uint32_t tP) {
+  const uint64_t c2 = f2_make(c, c);
+  const uint64_t nm2 = f2_make(-m_use, -m_use);
+  uint64_t la = f2_make(0.f, 0.f), lb = la;
+#pragma unroll
+  for (int ch = 0; ch < BN / 32; ++ch) {
+    // 32 columns -> 16 packed words -> tensor memory, chunk by chunk so that
+    // the registers of S are released as P is produced.
+    uint32_t pk[16];
+#pragma unroll
+    for (int w = 0; w < 16; ++w) {
+      const int k = ch * 32 + 2 * w;
+      const uint64_t x2 = f2_fma(f2_make(s[k], s[k + 1]), c2, nm2);
+      float x0, x1;
+      f2_split(x2, x0, x1);
+      const uint64_t e2 =
+          ((k & 7) < POLY8) ? ex2_poly2(x0, x1) : f2_make(ex2_approx(x0), ex2_approx(x1));
+      if (w & 1)
+        lb = f2_add(lb, e2);
+      else
+        la = f2_add(la, e2);
+      float e0, e1;
+      f2_split(e2, e0, e1);
+      pk[w] = pack2<T>(e0, e1);
+    }
+    tmem_st_x16(tP + ch * 16, pk);
+  }
+  float a0, a1, b0, b1;
+  f2_split(la, a0, a1);
+  f2_split(lb, b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+
+template <int D, typename T, bool CAUSAL, int POLY8, bool PINGPONG>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -137,54 +271,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem + C::kQOff;
   uint8_t* sKV = smem + C::kKVOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + S;
-  uint64_t* s_ready = kv_empty + S;
+  uint64_t* q_full = kv_empty + S;
+  uint64_t* q_empty = q_full + NQT;
+  uint64_t* s_ready = q_empty + NQT;
   uint64_t* p_ready = s_ready + NQT;
   uint64_t* o_done = p_ready + NQT;
-  uint64_t* drain = o_done + NQT;
+  uint64_t* turn = o_done + NQT;
+  uint64_t* drain = turn + NQT;
   CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem + C::kCtlOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kCtlOff + 32);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;  // b * Hq + h
-  const int b = bh / p.Hq;
-  const int h = bh - b * p.Hq;
-  const int kvh = h / p.group;
-  const int pair = CAUSAL ? (p.n_pairs - 1 - static_cast<int>(blockIdx.y))
-                          : static_cast<int>(blockIdx.y);
+  const int G = gridDim.x;
+  const int cta = blockIdx.x;
   const int nkv_all = (p.Nk + BN - 1) / BN;
 
-  // Key tiles each query tile needs (causal: stop at the last visible key).
-  int r0[NQT], nt[NQT];
-#pragma unroll
-  for (int t = 0; t < NQT; ++t) {
-    r0[t] = pair * (NQT * BM) + t * BM;
-    if (r0[t] >= p.Nq) {
-      nt[t] = 0;
-    } else if (!CAUSAL) {
-      nt[t] = nkv_all;
-    } else {
-      const int last_row = min(r0[t] + BM - 1, p.Nq - 1);
-      const long long kmax = static_cast<long long>(last_row) + p.off;
-      const long long ntiles = kmax / BN + 1;
-      nt[t] = kmax < 0 ? 0 : static_cast<int>(ntiles < nkv_all ? ntiles : nkv_all);
-    }
-  }
-  const int nmax = max(nt[0], nt[1]);
-
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
     for (int t = 0; t < NQT; ++t) {
+      mbar_init(&q_full[t], 1);
+      mbar_init(&q_empty[t], 1);
       mbar_init(&s_ready[t], 1);
       mbar_init(&p_ready[t], 4 * 32);
       mbar_init(&o_done[t], 1);
+      mbar_init(&turn[t], 4 * 32);
     }
     mbar_init(drain, 1);
     ctl->abort = 0;
@@ -207,100 +323,124 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && nmax > 0 && !(p.debug_flags & 1)) {
-      const int zkv = b * p.Hkv + kvh;
-      uint32_t qbytes = 0;
+    if (lane == 0 && !(p.debug_flags & 1)) {
+      uint32_t L = 0;       // K/V loads issued so far (K_j, V_j alternate)
+      int qn[NQT] = {0, 0};  // Q loads issued so far, per tile
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int idx = item_index(r, cta, G);
+        if (idx >= p.total) break;
+        const Item it = decode_item<CAUSAL>(idx, p, nkv_all);
 #pragma unroll
-      for (int t = 0; t < NQT; ++t)
-        if (r0[t] < p.Nq) qbytes += C::kTileBytes;
-      mbar_arrive_expect_tx(q_full, qbytes);
-#pragma unroll
-      for (int t = 0; t < NQT; ++t) {
-        if (r0[t] >= p.Nq) continue;
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d(sQ + t * C::kTileBytes + bx * C::kBoxBytes, &tm_q, q_full, bx * 64, r0[t],
-                      bh);
-      }
-      const int nloads = 2 * nmax;  // K_0, V_0, K_1, V_1, ...
-      int issued = 0;
-      for (int L = 0; L < nloads; ++L) {
-        const int s = L % S;
-        const int use = L / S;
-        if (use > 0 && !wait_bar(&kv_empty[s], (use - 1) & 1, ctl, kSiteKvEmpty)) break;
-        const CUtensorMap* map = (L & 1) ? &tm_v : &tm_k;
-        const int j = L >> 1;
-        mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d(sKV + s * C::kTileBytes + bx * C::kBoxBytes, map, &kv_full[s], bx * 64,
-                      j * BN, zkv);
-        issued = L + 1;
+        for (int t = 0; t < NQT; ++t) {
+          if ((t ? it.n1 : it.n0) == 0) continue;
+          if (qn[t] > 0 && !(ok = wait_bar(&q_empty[t], (qn[t] - 1) & 1, ctl, kSiteQEmpty)))
+            break;
+          mbar_arrive_expect_tx(&q_full[t], C::kTileBytes);
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d(sQ + t * C::kTileBytes + bx * C::kBoxBytes, &tm_q, &q_full[t], bx * 64,
+                        it.r0 + t * BM, it.bh);
+          ++qn[t];
+        }
+        const int nmax = max(it.n0, it.n1);
+        const int zkv = it.b * p.Hkv + it.kvh;
+        for (int l = 0; ok && l < 2 * nmax; ++l, ++L) {
+          const uint32_t s = L % S;
+          const uint32_t use = L / S;
+          if (use > 0 && !(ok = wait_bar(&kv_empty[s], (use - 1) & 1, ctl, kSiteKvEmpty))) break;
+          const CUtensorMap* map = (l & 1) ? &tm_v : &tm_k;
+          mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d(sKV + s * C::kTileBytes + bx * C::kBoxBytes, map, &kv_full[s], bx * 64,
+                        (l >> 1) * BN, zkv);
+        }
       }
       // No copy may still be landing in shared memory when the CTA exits.
-      drain_bar(q_full, 0, ctl, kSiteDrain);
-      for (int s = 0; s < S && s < issued; ++s) {
-        const int last = s + S * ((issued - 1 - s) / S);
-        drain_bar(&kv_full[s], (last / S) & 1, ctl, kSiteDrain);
+#pragma unroll
+      for (int t = 0; t < NQT; ++t)
+        if (qn[t] > 0) drain_bar(&q_full[t], (qn[t] - 1) & 1, ctl, kSiteDrain);
+      for (uint32_t s = 0; s < static_cast<uint32_t>(S) && s < L; ++s) {
+        const uint32_t cnt = (L - 1 - s) / S + 1;
+        drain_bar(&kv_full[s], (cnt - 1) & 1, ctl, kSiteDrain);
       }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nmax > 0) {
+    if (lane == 0) {
       constexpr uint32_t fmt = Fmt<T>::value;
       constexpr uint32_t idesc_s = umma_idesc_f16(fmt, BM, BN, 0, 0);
       constexpr uint32_t idesc_pv = umma_idesc_f16(fmt, BM, D, 0, 1);
       const uint32_t sq = smem_u32(sQ);
       const uint32_t skv = smem_u32(sKV);
-      bool ok = wait_bar(q_full, 0, ctl, kSiteQFull);
-      if (ok) tc_fence_after();
-      for (int j = 0; ok && j <= nmax; ++j) {
-        const int Lk = 2 * j;
-        const int Lv = 2 * j - 1;
-        bool have_k = false, have_v = false;
+      uint32_t L = 0;             // load index of K_0 of the current item
+      int qi[NQT] = {0, 0};       // items so far in which tile t had work
+      uint32_t pw[NQT] = {0, 0};  // p_ready phases consumed, per tile
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int idx = item_index(r, cta, G);
+        if (idx >= p.total) break;
+        const Item it = decode_item<CAUSAL>(idx, p, nkv_all);
+        const int nmax = max(it.n0, it.n1);
+        for (int j = 0; ok && j <= nmax; ++j) {
+          const uint32_t Lk = L + 2 * j;
+          const uint32_t Lv = L + 2 * j - 1;
+          bool have_k = false, have_v = false;
 #pragma unroll
-        for (int t = 0; t < NQT; ++t) {
-          if (!ok) break;
-          if (j >= 1 && j - 1 < nt[t]) {
-            // O_t += P_t(j-1) V_{j-1}
-            if (!have_v) {
-              ok = wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull);
-              if (!ok) break;
-              have_v = true;
-            }
-            ok = wait_bar(&p_ready[t], (j - 1) & 1, ctl, kSitePReady);
+          for (int t = 0; t < NQT; ++t) {
             if (!ok) break;
-            tc_fence_after();
-            const uint32_t vbase = skv + (Lv % S) * C::kTileBytes;
-            const uint32_t tP = tmem + t * BN + kPCol;
-            const uint32_t tO = tmem + C::kOCol + t * D;
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              const uint64_t bdesc = smem_desc_sw128(vbase + kk * 16 * 128, C::kBoxBytes, 1024);
-              umma_ts(tO, tP + kk * 8, bdesc, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
-            }
-            if (j - 1 == nt[t] - 1) umma_commit(&o_done[t]);
-          }
-          if (j < nt[t]) {
-            // S_t = Q_t K_j^T
-            if (!have_k) {
-              ok = wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull);
-              if (!ok) break;
+            const int n = t ? it.n1 : it.n0;
+            if (j >= 1 && j - 1 < n) {
+              // O_t (+)= P_t(j-1) V_{j-1}. The p_ready arrival for an item's
+              // first step comes after the softmax group read O_t of its
+              // previous item, so O_t is free to be overwritten here.
+              if (!have_v) {
+                if (!(ok = wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull))) break;
+                have_v = true;
+              }
+              if (!(ok = wait_bar(&p_ready[t], pw[t] & 1, ctl, kSitePReady))) break;
+              ++pw[t];
               tc_fence_after();
-              have_k = true;
-            }
-            const uint32_t kbase = skv + (Lk % S) * C::kTileBytes;
-            const uint32_t qbase = sq + t * C::kTileBytes;
-            const uint32_t tS = tmem + t * BN;
+              const uint32_t vbase = skv + (Lv % S) * C::kTileBytes;
+              const uint32_t tP = tmem + t * BN + kPCol;
+              const uint32_t tO = tmem + C::kOCol + t * D;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t koff = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-              umma_ss(tS, smem_desc_sw128(qbase + koff, 16, 1024),
-                      smem_desc_sw128(kbase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < BN / 16; ++kk) {
+                const uint64_t bdesc =
+                    smem_desc_sw128(vbase + kk * 16 * 128, C::kBoxBytes, 1024);
+                umma_ts(tO, tP + kk * 8, bdesc, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
+              }
+              if (j - 1 == n - 1) umma_commit(&o_done[t]);
             }
-            umma_commit(&s_ready[t]);
+            if (j < n) {
+              // S_t = Q_t K_j^T
+              if (!have_k) {
+                if (!(ok = wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull))) break;
+                tc_fence_after();
+                have_k = true;
+              }
+              if (j == 0) {
+                if (!(ok = wait_bar(&q_full[t], qi[t] & 1, ctl, kSiteQFull))) break;
+                tc_fence_after();
+              }
+              const uint32_t kbase = skv + (Lk % S) * C::kTileBytes;
+              const uint32_t qbase = sq + t * C::kTileBytes;
+              const uint32_t tS = tmem + t * BN;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+                umma_ss(tS, smem_desc_sw128(qbase + koff, 16, 1024),
+                        smem_desc_sw128(kbase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+              }
+              umma_commit(&s_ready[t]);
+              if (j == n - 1) umma_commit(&q_empty[t]);
+            }
           }
+          if (have_k) umma_commit(&kv_empty[Lk % S]);
+          if (have_v) umma_commit(&kv_empty[Lv % S]);
         }
-        if (have_k) umma_commit(&kv_empty[Lk % S]);
-        if (have_v) umma_commit(&kv_empty[Lv % S]);
+        L += 2 * nmax;
+        qi[0] += it.n0 > 0;
+        qi[1] += it.n1 > 0;
       }
       // Every MMA must be complete before tensor memory is released.
       umma_commit(drain);
@@ -310,117 +450,127 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;
     const int q4 = warp & 3;
-    const int rt = t ? r0[1] : r0[0];
-    const int row = rt + q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * BN;
     const uint32_t tP = tS + kPCol;
     const uint32_t tO = tmem + lane_off + C::kOCol + t * D;
     const float sl2 = p.scale_log2;
-    const int n = t ? nt[1] : nt[0];
-    float m = -INFINITY;  // running max of s * c (log2 units)
-    float l = 0.f;        // running sum of p
+    uint32_t sw = 0;  // s_ready phases consumed
+    uint32_t od = 0;  // o_done phases consumed
+    uint32_t tk = 0;  // turns taken
     bool ok = true;
-    for (int i = 0; i < n; ++i) {
-      ok = warp_all(wait_bar(&s_ready[t], i & 1, ctl, kSiteSReady));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t ra[32], rb[32], rc[32], rd[32];
-      tmem_ld_x32(tS + 0, ra);
-      tmem_ld_x32(tS + 32, rb);
-      tmem_ld_x32(tS + 64, rc);
-      tmem_ld_x32(tS + 96, rd);
-      tmem_wait_ld_x32(ra);
-      tmem_wait_ld_x32(rb);
-      tmem_wait_ld_x32(rc);
-      tmem_wait_ld_x32(rd);
-      float s[BN];
+    if (PINGPONG && t == 1) mbar_arrive(&turn[0]);  // tile 0 takes the first turn
+    for (int r = 0; ok; ++r) {
+      const int idx = item_index(r, cta, G);
+      if (idx >= p.total) break;
+      const Item it = decode_item<CAUSAL>(idx, p, nkv_all);
+      const int n = t ? it.n1 : it.n0;
+      const int rt = it.r0 + t * BM;
+      const int row = rt + q4 * 32 + lane;
+      float m = -INFINITY;  // running max of s * c (log2 units)
+      float l = 0.f;        // running sum of p
+      for (int i = 0; i < n; ++i) {
+        if (!(ok = warp_all(wait_bar(&s_ready[t], sw & 1, ctl, kSiteSReady)))) break;
+        ++sw;
+        tc_fence_after();
+        uint32_t ra[32], rb[32], rc[32], rd[32];
+        tmem_ld_x32(tS + 0, ra);
+        tmem_ld_x32(tS + 32, rb);
+        tmem_ld_x32(tS + 64, rc);
+        tmem_ld_x32(tS + 96, rd);
+        tmem_wait_ld_x32(ra);
+        tmem_wait_ld_x32(rb);
+        tmem_wait_ld_x32(rc);
+        tmem_wait_ld_x32(rd);
+        float s[BN];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        s[k] = __uint_as_float(ra[k]);
-        s[32 + k] = __uint_as_float(rb[k]);
-        s[64 + k] = __uint_as_float(rc[k]);
-        s[96 + k] = __uint_as_float(rd[k]);
-      }
-      const int kv0 = i * BN;
-      const bool edge = (CAUSAL && kv0 + BN - 1 > rt + p.off) || (kv0 + BN > p.Nk);
-      if (edge) {
-        const int last = (CAUSAL ? min(row + p.off, p.Nk - 1) : p.Nk - 1) - kv0;
-#pragma unroll
-        for (int k = 0; k < BN; ++k) s[k] = (k > last) ? -INFINITY : s[k];
-      }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-      for (int k = 4; k < BN; k += 4) {
-        mx0 = fmaxf(mx0, s[k]);
-        mx1 = fmaxf(mx1, s[k + 1]);
-        mx2 = fmaxf(mx2, s[k + 2]);
-        mx3 = fmaxf(mx3, s[k + 3]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-      float alpha = 1.f;
-      const bool need = m_tile > m + kRescaleThreshold;
-      if (need) {
-        alpha = ex2_approx(m - m_tile);  // m = -inf gives 0
-        m = m_tile;
-        l *= alpha;
-      }
-      const float m_use = (m == -INFINITY) ? 0.f : m;
-      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-      uint32_t pa[32], pb[32];
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        const float e0 = ex2_approx(fmaf(s[2 * c], sl2, -m_use));
-        const float e1 = ex2_approx(fmaf(s[2 * c + 1], sl2, -m_use));
-        const float e2 = ex2_approx(fmaf(s[2 * c + 2], sl2, -m_use));
-        const float e3 = ex2_approx(fmaf(s[2 * c + 3], sl2, -m_use));
-        l0 += e0;
-        l1 += e1;
-        l2 += e2;
-        l3 += e3;
-        pa[c] = pack2<T>(e0, e1);
-        pa[c + 1] = pack2<T>(e2, e3);
-      }
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        const float e0 = ex2_approx(fmaf(s[64 + 2 * c], sl2, -m_use));
-        const float e1 = ex2_approx(fmaf(s[64 + 2 * c + 1], sl2, -m_use));
-        const float e2 = ex2_approx(fmaf(s[64 + 2 * c + 2], sl2, -m_use));
-        const float e3 = ex2_approx(fmaf(s[64 + 2 * c + 3], sl2, -m_use));
-        l0 += e0;
-        l1 += e1;
-        l2 += e2;
-        l3 += e3;
-        pb[c] = pack2<T>(e0, e1);
-        pb[c + 1] = pack2<T>(e2, e3);
-      }
-      l += (l0 + l1) + (l2 + l3);
-      tmem_st_x32(tP, pa);
-      tmem_st_x32(tP + 32, pb);
-      if (i > 0 && __any_sync(0xffffffffu, need)) {
-        // O_t was last written by PV_t(i-1), complete before S_t(i) was signalled.
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld_x32(tO + c * 32, o);
-          tmem_wait_ld_x32(o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st_x32(tO + c * 32, o);
+        for (int k = 0; k < 32; ++k) {
+          s[k] = __uint_as_float(ra[k]);
+          s[32 + k] = __uint_as_float(rb[k]);
+          s[64 + k] = __uint_as_float(rc[k]);
+          s[96 + k] = __uint_as_float(rd[k]);
         }
+        const int kv0 = i * BN;
+        const bool edge = (CAUSAL && kv0 + BN - 1 > rt + p.off) || (kv0 + BN > p.Nk);
+        if (edge) {
+          const int last = (CAUSAL ? min(row + p.off, p.Nk - 1) : p.Nk - 1) - kv0;
+#pragma unroll
+          for (int k = 0; k < BN; ++k) s[k] = (k > last) ? -INFINITY : s[k];
+        }
+        // four independent chains of 3-input max, 32 columns each
+        float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[32], s[33]);
+        float mx2 = fmaxf(s[64], s[65]), mx3 = fmaxf(s[96], s[97]);
+#pragma unroll
+        for (int k = 2; k < 32; k += 2) {
+          mx0 = fmax3(mx0, s[k], s[k + 1]);
+          mx1 = fmax3(mx1, s[32 + k], s[33 + k]);
+          mx2 = fmax3(mx2, s[64 + k], s[65 + k]);
+          mx3 = fmax3(mx3, s[96 + k], s[97 + k]);
+        }
+        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        float alpha = 1.f;
+        const bool need = m_tile > m + kRescaleThreshold;
+        if (need) {
+          alpha = ex2_approx(m - m_tile);  // m = -inf gives 0
+          m = m_tile;
+          l *= alpha;
+        }
+        const float m_use = (m == -INFINITY) ? 0.f : m;
+        if (PINGPONG) {
+          if (!(ok = warp_all(wait_bar(&turn[t], tk & 1, ctl, kSiteTurn)))) break;
+          ++tk;
+        }
+        float lsum;
+        if (POLY8 > 0 && !edge)
+          lsum = exp_tile<T, POLY8>(s, sl2, m_use, tP);
+        else
+          lsum = exp_tile<T, 0>(s, sl2, m_use, tP);
+        l += lsum;
+        if (PINGPONG) mbar_arrive(&turn[t ^ 1]);
+        if (i > 0 && __any_sync(0xffffffffu, need)) {
+          // O_t was last written by PV_t(i-1), complete before S_t(i) was signalled.
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_x32(tO + c * 32, o);
+            tmem_wait_ld_x32(o);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float a0, a1;
+              f2_split(f2_mul(f2_make(__uint_as_float(o[e]), __uint_as_float(o[e + 1])),
+                              f2_make(alpha, alpha)),
+                       a0, a1);
+              o[e] = __float_as_uint(a0);
+              o[e + 1] = __float_as_uint(a1);
+            }
+            tmem_st_x32(tO + c * 32, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_ready[t]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_ready[t]);
-    }
-    if (ok && n > 0) {
-      ok = warp_all(wait_bar(&o_done[t], 0, ctl, kSiteODone));
-      if (ok) tc_fence_after();
-    }
-    if (ok) {
+      if (!ok) break;
+      if (PINGPONG) {
+        // Keep the turn order in step with the other group: each group takes
+        // max(n0, n1) turns per item.
+        const int nturns = max(it.n0, it.n1);
+        for (int i = n; i < nturns; ++i) {
+          if (!(ok = warp_all(wait_bar(&turn[t], tk & 1, ctl, kSiteTurn)))) break;
+          ++tk;
+          mbar_arrive(&turn[t ^ 1]);
+        }
+        if (!ok) break;
+      }
+      if (rt >= p.Nq) continue;  // no rows in this tile
+      if (n > 0) {
+        if (!(ok = warp_all(wait_bar(&o_done[t], od & 1, ctl, kSiteODone)))) break;
+        ++od;
+        tc_fence_after();
+      }
       const bool has_row = row < p.Nq;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<size_t>(bh) * p.Nq + row) * D;
+      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<size_t>(it.bh) * p.Nq + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -433,8 +583,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack2<T>(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        for (int e = 0; e < 16; ++e) {
+          float a0, a1;
+          f2_split(f2_mul(f2_make(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])),
+                          f2_make(inv_l, inv_l)),
+                   a0, a1);
+          w[e] = pack2<T>(a0, a1);
+        }
         if (has_row) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
           dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -444,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (has_row && p.lse != nullptr) {
-        p.lse[static_cast<size_t>(bh) * p.Nq + row] =
+        p.lse[static_cast<size_t>(it.bh) * p.Nq + row] =
             l > 0.f ? (m + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
       }
     }
