@@ -28,7 +28,7 @@ __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, CtaCtl* ct
   const uint64_t t0 = globaltimer_ns();
   volatile int* abort = &ctl->abort;
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     if ((n & 15u) == 0) {
       if (honour_abort && *abort) return false;
       if (globaltimer_ns() - t0 > ctl->wait_ns) {
@@ -42,10 +42,14 @@ __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, CtaCtl* ct
 
 // Wait until the phase with the given parity of `bar` has completed. Returns
 // false (without completing) when the CTA is aborting or the time limit passed.
+// The first poll sleeps in try_wait with a suspend-time hint, so a waiting
+// thread takes no issue slots from its neighbours and is woken as soon as the
+// phase completes; only if that poll times out does the wait read the global
+// timer (a slow read) and start checking the time limit.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, CtaCtl* ctl,
                                          unsigned site) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  if (mbar_try_wait_sleep(a, parity)) return true;
   return wait_slow(a, parity, ctl, site, true);
 }
 
