@@ -8,8 +8,9 @@ One step = one pass of the whole path over one batch of synthetic input:
 `value` is the prefill throughput in TFLOP/s (algorithmic FLOPs: 4*d per
 visible query/key pair) over the prefill kernel's CUDA-event time, summed over
 ranks (weak scaling: every rank runs its own batch). The decode side is
-reported in the `decode` object in GB/s of KV cache read. L2 is flushed (a
-256 MiB write) before every step; the flush is outside the kernel events.
+reported in the `decode` object in GB/s of KV cache read. L2 is flushed before
+every step (a 256 MiB write, then a 256 MiB read that evicts the written lines);
+the flush is outside the kernel events.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -348,12 +349,20 @@ def run_ours(args, world, rank, local):
                                                 seed=DECODE.seed + seed_off)
     do = torch.empty_like(dq)
     dlse = torch.empty(DECODE.B, DECODE.Hq, device=dev, dtype=torch.float32)
-    flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)  # 256 MiB > L2
+    # L2 flush between steps: write 256 MiB (> 126 MB L2), then read another
+    # 256 MiB so that the dirty lines of the write are evicted (written back)
+    # before the timed kernels start rather than during them.
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)
+    flush_rd = torch.zeros(64 * 1024 * 1024, dtype=torch.int32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        flush_rd.max()
 
     stream = torch.cuda.current_stream()
 
     def step(evs=None):
-        flush.zero_()
+        flush_l2()
         if evs:
             evs[0].record(stream)
         eta.attn_fwd(q, k, v, o=o, lse=lse, scale=PREFILL.scale, causal=True, stream=stream)
@@ -459,7 +468,8 @@ def run_ours(args, world, rank, local):
                        "kv_tokens": int(sl_cpu.sum()), "kv_bytes": kv_bytes,
                        "nsplit": eta.attn_decode_num_splits(DECODE.B, DECODE.Hq, DECODE.Hkv,
                                                             DECODE.d)},
-            "l2": "flushed before every step (256 MiB write, outside the kernel events)",
+            "l2": "flushed before every step (256 MiB write, then a 256 MiB read that "
+                  "evicts its dirty lines; outside the kernel events)",
             "parallelism": f"replicas x{world} (independent batches per GPU)",
         },
         "roofline": {"bound": "tensor", "achieved": pre_ach, "peak": peaks["bf16_tflops"],

@@ -179,14 +179,19 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                 : launch_prefill<64, T, false>(tq, tk, tv, p, grid, st);
 }
 
-// Split-KV count: enough CTAs for about eight waves of resident split CTAs.
+// Split-KV count: enough CTAs for about ETA_DECODE_WAVES waves of resident
+// split CTAs (3 resident per SM), at most 64 splits.
+#ifndef ETA_DECODE_WAVES
+#define ETA_DECODE_WAVES 8
+#endif
 int decode_splits(int B, int Hq, int Hkv, int d, int sm_count) {
+  (void)d;
   const int G = Hq / Hkv;
   const int GP = G <= 4 ? 4 : 8;
   const int nchunk = (G + GP - 1) / GP;
   const long long units = static_cast<long long>(B) * Hkv * nchunk;
-  const int resident = (d == 128 ? 3 : 3) * sm_count;
-  long long ns = units > 0 ? (8LL * resident + units - 1) / units : 1;
+  const long long resident = 3LL * sm_count;
+  long long ns = units > 0 ? (ETA_DECODE_WAVES * resident + units - 1) / units : 1;
   if (ns < 1) ns = 1;
   if (ns > 64) ns = 64;
   return static_cast<int>(ns);

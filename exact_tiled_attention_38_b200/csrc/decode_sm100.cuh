@@ -7,14 +7,16 @@
 // "Reduced IO Is Not the Same as Eliminating KV Cache" section: the cache still
 // has to be read). The kernel therefore streams each byte of K and V once:
 //
-//   split pass   grid (nsplit, Hkv * head chunks, B), 128 threads. A CTA takes
-//                a contiguous chunk of one sequence's keys for one KV head,
-//                copies it into shared memory with bulk asynchronous copies
-//                (a 4-stage ring of 32-key K and V blocks), and computes, for
-//                the query heads sharing that KV head, the scores (16-byte
-//                vector reads, butterfly shuffle reductions), a running
-//                softmax and the weighted sum of V. It writes the chunk's
-//                normalised partial output and its log-sum-exp (log2 units).
+//   split pass   grid (nsplit, Hkv * head chunks, B); 4 consumer warps and one
+//                producer warp. A CTA takes a contiguous chunk of one
+//                sequence's keys for one KV head; the producer copies it into
+//                shared memory with bulk asynchronous copies (a ring of 32-key
+//                K and V blocks with full/empty mbarriers, so no warp waits for
+//                another), and the consumers compute, for the query heads
+//                sharing that KV head, the scores (16-byte vector reads, fp32
+//                pair FMAs, butterfly shuffle reductions), a running softmax and
+//                the weighted sum of V. It writes the chunk's normalised
+//                partial output and its log-sum-exp (log2 units).
 //   combine      one warp per (b, query head): merges the partials by their
 //                log-sum-exp and writes O (input dtype) and LSE (natural log).
 //
@@ -34,11 +36,18 @@
 namespace eta {
 namespace decode {
 
-constexpr int kThreads = 128;
-constexpr int kWarps = 4;
+__device__ __forceinline__ bool warp_all_d(bool v) { return __all_sync(0xffffffffu, v); }
+
+constexpr int kWarps = 4;                     // consumer warps
+constexpr int kThreads = 32 * (kWarps + 1);   // + one producer warp
 constexpr float kRescaleThreshold = 8.0f;
 
 enum : unsigned { kSiteStage = 0x21, kSiteDrain = 0x22 };
+
+// Ring depth in 32-key stages (d = 128; twice as many for d = 64).
+#ifndef ETA_DECODE_STAGES
+#define ETA_DECODE_STAGES 3
+#endif
 
 // GP: query heads per CTA (the group, padded up to 4 or 8).
 template <int D, int GP>
@@ -54,9 +63,9 @@ struct DCfg {
   static constexpr int kRowBytes = D * 2;
   static constexpr int kHalfBytes = TK * kRowBytes;  // K (or V) block of one stage
   static constexpr int kStageBytes = 2 * kHalfBytes;
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kStages = (D == 128) ? ETA_DECODE_STAGES : 2 * ETA_DECODE_STAGES;
   static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kCtlOff = kBarOff + kStages * 8;
+  static constexpr int kCtlOff = kBarOff + 2 * kStages * 8;  // full[S], empty[S]
   static constexpr int kXOff = kCtlOff + 32;             // per-warp exchange: 32 p + GP alpha
   static constexpr int kMiscOff = kXOff + kWarps * 64 * 4;
   static constexpr int kSmemBytes = kMiscOff + 32;
@@ -82,31 +91,6 @@ struct DParams {
 };
 
 template <typename T>
-__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]);
-
-template <>
-__device__ __forceinline__ void unpack8<__nv_bfloat16>(const uint4& v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
-template <>
-__device__ __forceinline__ void unpack8<__half>(const uint4& v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2 h2 = *reinterpret_cast<const __half2*>(&w[i]);
-    const float2 x = __half22float2(h2);
-    f[2 * i] = x.x;
-    f[2 * i + 1] = x.y;
-  }
-}
-
-template <typename T>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi);
 template <>
 __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
@@ -119,6 +103,28 @@ __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// bf16/fp16 x8 (one 16-byte chunk) -> four fp32 pairs.
+template <typename T>
+__device__ __forceinline__ void unpack8x2(const uint4& v, uint64_t (&f)[4]);
+
+template <>
+__device__ __forceinline__ void unpack8x2<__nv_bfloat16>(const uint4& v, uint64_t (&f)[4]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    f[i] = f2_make(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+
+template <>
+__device__ __forceinline__ void unpack8x2<__half>(const uint4& v, uint64_t (&f)[4]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    f[i] = f2_make(x.x, x.y);
+  }
+}
+
 template <int D, int GP, typename T>
 __global__ void __launch_bounds__(kThreads) attn_decode_split_kernel(const DParams p) {
   using C = DCfg<D, GP>;
@@ -127,6 +133,7 @@ __global__ void __launch_bounds__(kThreads) attn_decode_split_kernel(const DPara
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* empty = full + S;
   CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem + C::kCtlOff);
   float* xch = reinterpret_cast<float*>(smem + C::kXOff);
   long long* misc = reinterpret_cast<long long*>(smem + C::kMiscOff);
@@ -150,8 +157,11 @@ __global__ void __launch_bounds__(kThreads) attn_decode_split_kernel(const DPara
       misc[1] = max(p.seqlens[b], 0);
     }
   }
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kWarps);
+    }
     ctl->abort = 0;
     ctl->wait_ns = p.wait_ns;
     fence_mbar_init();
@@ -169,75 +179,85 @@ __global__ void __launch_bounds__(kThreads) attn_decode_split_kernel(const DPara
   const T* kbase = reinterpret_cast<const T*>(p.kc) + head_base;
   const T* vbase = reinterpret_cast<const T*>(p.vc) + head_base;
 
-  // Query rows of this CTA's heads, pre-scaled by scale * log2 e.
-  float qr[GP][8];
-#pragma unroll
-  for (int hh = 0; hh < GP; ++hh) {
-    const int gi = hc * GP + hh;
-    if (gi < p.G) {
-      const int hq = g * p.G + gi;
-      const uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
-                                                        (static_cast<size_t>(b) * p.Hq + hq) * D +
-                                                        li * 8);
-      unpack8<T>(raw, qr[hh]);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) qr[hh][c] *= p.scale_log2;
-    } else {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) qr[hh][c] = 0.f;
-    }
-  }
-
-  auto issue = [&](int it) {
-    const int s = it % S;
-    const int t0 = t_begin + it * TK;
-    const int nk = min(TK, t_end - t0);
-    const uint32_t bytes = static_cast<uint32_t>(nk) * C::kRowBytes;
-    uint8_t* dst = stages + s * C::kStageBytes;
-    mbar_arrive_expect_tx(&full[s], 2 * bytes);
-    bulk_load(dst, kbase + static_cast<size_t>(t0) * D, bytes, &full[s]);
-    bulk_load(dst + C::kHalfBytes, vbase + static_cast<size_t>(t0) * D, bytes, &full[s]);
-  };
-  int issued = 0;
-  if (threadIdx.x == 0) {
-    for (int it = 0; it < n_iter && it < S; ++it) issue(it);
-    issued = min(n_iter, S);
-  }
-
   float m_run = -INFINITY;  // running max for head (li % GP), log2 units
   float l_lane = 0.f;       // this lane's share of the running sum for that head
-  float o[GP][8];
-#pragma unroll
-  for (int hh = 0; hh < GP; ++hh)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) o[hh][c] = 0.f;
-  float* xw = xch + warp * 64;
+  uint64_t o2[GP][4];       // output accumulators, fp32 pairs (8 dims per lane)
 
-  for (int it = 0; it < n_iter; ++it) {
-    const int s = it % S;
-    const bool ok = wait_bar(&full[s], (it / S) & 1, ctl, kSiteStage);
-    if (ok) {
+  if (warp == kWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < n_iter; ++it) {
+        const int s = it % S;
+        const int use = it / S;
+        if (use > 0 && !wait_bar(&empty[s], (use - 1) & 1, ctl, kSiteStage)) break;
+        const int t0 = t_begin + it * TK;
+        const int nk = min(TK, t_end - t0);
+        const uint32_t bytes = static_cast<uint32_t>(nk) * C::kRowBytes;
+        uint8_t* dst = stages + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], 2 * bytes);
+        bulk_load(dst, kbase + static_cast<size_t>(t0) * D, bytes, &full[s]);
+        bulk_load(dst + C::kHalfBytes, vbase + static_cast<size_t>(t0) * D, bytes, &full[s]);
+        issued = it + 1;
+      }
+      // No bulk copy may still be landing when the stages are reused or the CTA exits.
+      for (int s = 0; s < S && s < issued; ++s) {
+        const int last = s + S * ((issued - 1 - s) / S);
+        drain_bar(&full[s], (last / S) & 1, ctl, kSiteDrain);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    // Query rows of this CTA's heads, pre-scaled by scale * log2 e.
+    uint64_t qr[GP][4];
+#pragma unroll
+    for (int hh = 0; hh < GP; ++hh) {
+      const int gi = hc * GP + hh;
+      if (gi < p.G) {
+        const int hq = g * p.G + gi;
+        const uint4 raw = *reinterpret_cast<const uint4*>(
+            reinterpret_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + hq) * D + li * 8);
+        unpack8x2<T>(raw, qr[hh]);
+        const uint64_t sc2 = f2_make(p.scale_log2, p.scale_log2);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qr[hh][c] = f2_mul(qr[hh][c], sc2);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qr[hh][c] = f2_make(0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < GP; ++hh)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) o2[hh][c] = f2_make(0.f, 0.f);
+    float* xw = xch + warp * 64;
+    for (int it = 0; it < n_iter; ++it) {
+      const int s = it % S;
+      if (!warp_all_d(wait_bar(&full[s], (it / S) & 1, ctl, kSiteStage))) break;
       const int nk = min(TK, t_end - (t_begin + it * TK));
       const uint8_t* ks = stages + s * C::kStageBytes;
       const uint8_t* vs = ks + C::kHalfBytes;
 #pragma unroll
       for (int bb = 0; bb < BPS; ++bb) {
         const int rbase = (warp * BPS + bb) * R;
-        // scores: partial dot products over this lane's 8 dims, then a
-        // butterfly reduce-scatter over the LPR lanes of the row group.
+        // scores: partial dot products over this lane's 8 dims (fp32 pairs),
+        // then a butterfly reduce-scatter over the LPR lanes of the row group.
         float v[LPR];
 #pragma unroll
         for (int mm = 0; mm < RB; ++mm) {
           const int r = rbase + grp + NGRP * mm;
           const uint4 raw = *reinterpret_cast<const uint4*>(ks + r * C::kRowBytes + li * 16);
-          float kf[8];
-          unpack8<T>(raw, kf);
+          uint64_t kf[4];
+          unpack8x2<T>(raw, kf);
 #pragma unroll
           for (int hh = 0; hh < GP; ++hh) {
-            float acc = qr[hh][0] * kf[0];
-#pragma unroll
-            for (int c = 1; c < 8; ++c) acc = fmaf(qr[hh][c], kf[c], acc);
-            v[mm * GP + hh] = acc;
+            uint64_t acc = f2_mul(qr[hh][0], kf[0]);
+            acc = f2_fma(qr[hh][1], kf[1], acc);
+            acc = f2_fma(qr[hh][2], kf[2], acc);
+            acc = f2_fma(qr[hh][3], kf[3], acc);
+            float a0, a1;
+            f2_split(acc, a0, a1);
+            v[mm * GP + hh] = a0 + a1;
           }
         }
 #pragma unroll
@@ -273,73 +293,71 @@ __global__ void __launch_bounds__(kThreads) attn_decode_split_kernel(const DPara
 #pragma unroll
           for (int hh = 0; hh < GP; ++hh) {
             const float a = xw[32 + hh];
+            const uint64_t a2 = f2_make(a, a);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) o[hh][c] *= a;
+            for (int c = 0; c < 4; ++c) o2[hh][c] = f2_mul(o2[hh][c], a2);
           }
         }
 #pragma unroll
         for (int mm = 0; mm < RB; ++mm) {
           const int r = rbase + grp + NGRP * mm;
-          float vf[8];
+          uint64_t vf[4];
           if (r < nk) {
             const uint4 raw = *reinterpret_cast<const uint4*>(vs + r * C::kRowBytes + li * 16);
-            unpack8<T>(raw, vf);
+            unpack8x2<T>(raw, vf);
           } else {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) vf[c] = 0.f;
+            for (int c = 0; c < 4; ++c) vf[c] = f2_make(0.f, 0.f);
           }
           const float* pw = xw + grp * LPR + mm * GP;
 #pragma unroll
           for (int hh = 0; hh < GP; ++hh) {
             const float pm = pw[hh];
+            const uint64_t p2 = f2_make(pm, pm);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) o[hh][c] = fmaf(pm, vf[c], o[hh][c]);
+            for (int c = 0; c < 4; ++c) o2[hh][c] = f2_fma(p2, vf[c], o2[hh][c]);
           }
         }
         __syncwarp();
       }
+      // this warp is done with the stage
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
-    if (__syncthreads_or(!ok)) break;
-    if (threadIdx.x == 0 && it + S < n_iter) {
-      issue(it + S);
-      issued = it + S + 1;
-    }
-  }
-  // No bulk copy may still be landing when the stages are reused or the CTA exits.
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S && s < issued; ++s) {
-      const int last = s + S * ((issued - 1 - s) / S);
-      drain_bar(&full[s], (last / S) & 1, ctl, kSiteDrain);
-    }
-  }
-
-  // Merge the row groups of each warp, then the warps of the CTA.
-#pragma unroll
-  for (int M = LPR; M < 32; M <<= 1)
-#pragma unroll
-    for (int hh = 0; hh < GP; ++hh)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) o[hh][c] += __shfl_xor_sync(0xffffffffu, o[hh][c], M);
-  float lt = l_lane;
-#pragma unroll
-  for (int M = GP; M < 32; M <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, M);
-
-  __syncthreads();
-  float* red_m = reinterpret_cast<float*>(stages);  // [warps][GP]
-  float* red_l = red_m + kWarps * GP;               // [warps][GP]
-  float* red_o = red_l + kWarps * GP;               // [warps][GP][D]
-  if (grp == 0 && li < GP) {
-    red_m[warp * GP + li] = m_run;
-    red_l[warp * GP + li] = lt;
-  }
-  if (grp == 0) {
-#pragma unroll
-    for (int hh = 0; hh < GP; ++hh)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) red_o[(warp * GP + hh) * D + li * 8 + c] = o[hh][c];
   }
   __syncthreads();
   if (ctl->abort) return;
+
+  // Merge the row groups of each warp, then the warps of the CTA.
+  float* red_m = reinterpret_cast<float*>(stages);  // [warps][GP]
+  float* red_l = red_m + kWarps * GP;               // [warps][GP]
+  float* red_o = red_l + kWarps * GP;               // [warps][GP][D]
+  if (warp < kWarps) {
+    float o[GP][8];
+#pragma unroll
+    for (int hh = 0; hh < GP; ++hh)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) f2_split(o2[hh][c], o[hh][2 * c], o[hh][2 * c + 1]);
+#pragma unroll
+    for (int M = LPR; M < 32; M <<= 1)
+#pragma unroll
+      for (int hh = 0; hh < GP; ++hh)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) o[hh][c] += __shfl_xor_sync(0xffffffffu, o[hh][c], M);
+    float lt = l_lane;
+#pragma unroll
+    for (int M = GP; M < 32; M <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, M);
+    if (grp == 0 && li < GP) {
+      red_m[warp * GP + li] = m_run;
+      red_l[warp * GP + li] = lt;
+    }
+    if (grp == 0) {
+#pragma unroll
+      for (int hh = 0; hh < GP; ++hh)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) red_o[(warp * GP + hh) * D + li * 8 + c] = o[hh][c];
+    }
+  }
+  __syncthreads();
   for (int idx = threadIdx.x; idx < GP * D; idx += kThreads) {
     const int hh = idx / D;
     const int dim = idx - hh * D;

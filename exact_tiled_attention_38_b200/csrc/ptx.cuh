@@ -56,8 +56,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 #define ETA_SUSPEND_HINT_NS 1000000
 #endif
 // try_wait with a suspend-time hint: the thread sleeps until the phase
-// completes (it is woken then) or the hint in nanoseconds passes.
+// completes (it is woken then) or the hint in nanoseconds passes. A hint of 0
+// selects the plain form (system-dependent suspend time).
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+#if ETA_SUSPEND_HINT_NS > 0
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -67,6 +69,9 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
       : "r"(bar), "r"(parity), "n"(ETA_SUSPEND_HINT_NS)
       : "memory");
   return ok != 0;
+#else
+  return mbar_try_wait(bar, parity);
+#endif
 }
 
 // ---------------------------------------------------------------- TMA
