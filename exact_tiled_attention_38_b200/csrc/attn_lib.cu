@@ -67,16 +67,17 @@ inline bool aligned(const void* p, uintptr_t a) {
 
 inline bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 
-// 3-D map over a [Z][rows][D] tensor of 16-bit elements, box 64 x 128 x 1,
-// 128-byte swizzle, zero fill outside the tensor.
-int encode_3d(CUtensorMap* map, const void* base, bool bf16, int D, long long rows, long long Z) {
+// 3-D map over a [Z][rows][D] tensor of 16-bit elements, box 64 x box_rows x 1,
+// 128-byte swizzle, zero fill outside the tensor (loads) / clipping (stores).
+int encode_3d(CUtensorMap* map, const void* base, bool bf16, int D, long long rows, long long Z,
+              unsigned box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return ATTN_ERR_CUDA;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(Z)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                                  static_cast<cuuint64_t>(rows) * D * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                         3, const_cast<void*>(base), dims, strides, box, estr,
@@ -114,7 +115,7 @@ int launch_fill_empty(void* o, float* lse, long long rows, int D, cudaStream_t s
 
 template <int D, typename T, bool CAUSAL>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const prefill::Params& p, int grid, cudaStream_t st) {
+                   const CUtensorMap& to, const prefill::Params& p, int grid, cudaStream_t st) {
   auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, ETA_PREFILL_POLY8, false>;
   constexpr int smem = prefill::Cfg<D>::kSmemBytes;
   static std::once_flag once;
@@ -123,7 +124,7 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return ATTN_ERR_CUDA;
-  kern<<<grid, prefill::kThreads, smem, st>>>(tq, tk, tv, p);
+  kern<<<grid, prefill::kThreads, smem, st>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -148,8 +149,9 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   if (Nk == 0) return launch_fill_empty<T>(o, lse, static_cast<long long>(B) * Hq * Nq, d, st);
 
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   int rc = encode_3d(&tq, q, bf16, d, Nq, static_cast<long long>(B) * Hq);
+  if (rc == ATTN_OK) rc = encode_3d(&to, o, bf16, d, Nq, static_cast<long long>(B) * Hq, 32);
   if (rc == ATTN_OK) rc = encode_3d(&tk, k, bf16, d, Nk, static_cast<long long>(B) * Hkv);
   if (rc == ATTN_OK) rc = encode_3d(&tv, v, bf16, d, Nk, static_cast<long long>(B) * Hkv);
   if (rc != ATTN_OK) return rc;
@@ -173,10 +175,10 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   p.debug_flags = debug_flags;
   const int grid = static_cast<int>(total < info.sm_count ? total : info.sm_count);
   if (d == 128)
-    return causal ? launch_prefill<128, T, true>(tq, tk, tv, p, grid, st)
-                  : launch_prefill<128, T, false>(tq, tk, tv, p, grid, st);
-  return causal ? launch_prefill<64, T, true>(tq, tk, tv, p, grid, st)
-                : launch_prefill<64, T, false>(tq, tk, tv, p, grid, st);
+    return causal ? launch_prefill<128, T, true>(tq, tk, tv, to, p, grid, st)
+                  : launch_prefill<128, T, false>(tq, tk, tv, to, p, grid, st);
+  return causal ? launch_prefill<64, T, true>(tq, tk, tv, to, p, grid, st)
+                : launch_prefill<64, T, false>(tq, tk, tv, to, p, grid, st);
 }
 
 // Split-KV count: enough CTAs for about ETA_DECODE_WAVES waves of resident

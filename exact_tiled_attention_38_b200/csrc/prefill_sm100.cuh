@@ -86,13 +86,17 @@ struct Cfg {
   static constexpr int kStages = (D == 128) ? 4 : 6;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = NQT * kTileBytes;
-  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  // O staging for the TMA-store epilogue: per softmax warp 32 rows x 64 columns.
+  static constexpr int kStgWarpBytes = 32 * 128;
+  static constexpr int kStgOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kStgOff + 8 * kStgWarpBytes;
   // kv_full[S], kv_empty[S], then per tile: q_full, q_empty, s_ready, p_ready,
   // o_done, turn; then drain.
   static constexpr int kNumBars = 2 * kStages + 6 * NQT + 1;
   static constexpr int kCtlOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kCtlOff + 64 + 1024;  // + runtime 1024-byte alignment
   static constexpr uint32_t kOCol = 2 * BN;
+  static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 struct Params {
@@ -139,6 +143,11 @@ struct Fmt<__half> {
 };
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+// Make this thread's shared-memory writes visible to the async proxy (TMA).
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 // 2^x on the FMA and integer pipes, for x <= 8.
 // Range reduction: n = round(x) (adding 1.5 * 2^23 leaves round(x) in the low
@@ -261,7 +270,8 @@ template <int D, typename T, bool CAUSAL, int POLY8, bool PINGPONG>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_o, const Params p) {
   using C = Cfg<D>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -315,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
   }
   tc_fence_before();
   __syncthreads();
@@ -454,6 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_off + t * BN;
     const uint32_t tP = tS + kPCol;
     const uint32_t tO = tmem + lane_off + C::kOCol + t * D;
+    uint8_t* stg = smem + C::kStgOff + warp * C::kStgWarpBytes;  // this warp's O staging
     const float sl2 = p.scale_log2;
     uint32_t sw = 0;  // s_ready phases consumed
     uint32_t od = 0;  // o_done phases consumed
@@ -570,32 +582,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const bool has_row = row < p.Nq;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<size_t>(it.bh) * p.Nq + row) * D;
+      // O in 64-column halves: each lane packs its row's 64 columns into this
+      // warp's staging buffer (32 rows x 128 bytes, 128-byte swizzle: 16-byte
+      // chunk g of row lane sits at chunk position g ^ (lane % 8)), and one TMA
+      // store per half writes the 32 x 64 box (rows past Nq are clipped).
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (n > 0) {
-          tmem_ld_x32(tO + c * 32, o);
-          tmem_wait_ld_x32(o);
-        } else {
+      for (int half = 0; half < D / 64; ++half) {
+        if (lane == 0) bulk_wait_group_read0();  // the buffer's previous store has read it
+        __syncwarp();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = half * 2 + cc;
+          uint32_t o[32];
+          if (n > 0) {
+            tmem_ld_x32(tO + c * 32, o);
+            tmem_wait_ld_x32(o);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float a0, a1;
+            f2_split(f2_mul(f2_make(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])),
+                            f2_make(inv_l, inv_l)),
+                     a0, a1);
+            w[e] = pack2<T>(a0, a1);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int g = cc * 4 + j;
+            uint4* dst = reinterpret_cast<uint4*>(stg + lane * 128 + ((g ^ (lane & 7)) << 4));
+            *dst = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          }
         }
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float a0, a1;
-          f2_split(f2_mul(f2_make(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])),
-                          f2_make(inv_l, inv_l)),
-                   a0, a1);
-          w[e] = pack2<T>(a0, a1);
-        }
-        if (has_row) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
-          dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
+        fence_async_smem();
+        __syncwarp();
+        const int y = rt + q4 * 32;
+        if (lane == 0 && y < p.Nq) {
+          tma_store_3d(&tm_o, stg, half * 64, y, it.bh);
+          bulk_commit_group();
         }
       }
       if (has_row && p.lse != nullptr) {
@@ -605,6 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if (warp < 8 && lane == 0) bulk_wait_group0();  // stores of O done before the CTA exits
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
