@@ -17,7 +17,8 @@
 // Warp roles (320 threads):
 //   warps 0-3  softmax for query tile 0 (one thread per query row)
 //   warps 4-7  softmax for query tile 1
-//   warp  8    tensor-memory owner and the single thread that issues tcgen05.mma
+//   warp  8    tensor-memory owner; runs the MMA issue loop as a whole warp,
+//              one elected lane issuing each tcgen05.mma
 //   warp  9    TMA producer: Q tiles, then K_j and V_j through a ring of stages
 // Tensor memory (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256),
 // O_0 [256, 256+D), O_1 [256+D, 256+2D); the bf16/fp16 probabilities P_t
@@ -377,86 +378,99 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t fmt = Fmt<T>::value;
-      constexpr uint32_t idesc_s = umma_idesc_f16(fmt, BM, BN, 0, 0);
-      constexpr uint32_t idesc_pv = umma_idesc_f16(fmt, BM, D, 0, 1);
-      const uint32_t sq = smem_u32(sQ);
-      const uint32_t skv = smem_u32(sKV);
-      uint32_t L = 0;             // load index of K_0 of the current item
-      int qi[NQT] = {0, 0};       // items so far in which tile t had work
-      uint32_t pw[NQT] = {0, 0};  // p_ready phases consumed, per tile
-      bool ok = true;
-      for (int r = 0; ok; ++r) {
-        const int idx = item_index(r, cta, G);
-        if (idx >= p.total) break;
-        const Item it = decode_item<CAUSAL>(idx, p, nkv_all);
-        const int nmax = max(it.n0, it.n1);
-        for (int j = 0; ok && j <= nmax; ++j) {
-          const uint32_t Lk = L + 2 * j;
-          const uint32_t Lv = L + 2 * j - 1;
-          bool have_k = false, have_v = false;
+    // The whole warp runs this loop, so the descriptor arithmetic stays
+    // warp-uniform; one elected lane issues each tcgen05 instruction.
+    // Descriptors are built once and stepped by adding to the address field of
+    // their low word; Q and K are K-major, V is MN-major with its two
+    // 64-column halves kBoxBytes apart, and all share the high word.
+    constexpr uint32_t fmt = Fmt<T>::value;
+    constexpr uint32_t idesc_s = umma_idesc_f16(fmt, BM, BN, 0, 0);
+    constexpr uint32_t idesc_pv = umma_idesc_f16(fmt, BM, D, 0, 1);
+    const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+    const uint32_t d_hi = static_cast<uint32_t>(dq >> 32);
+    const uint32_t q_lo = static_cast<uint32_t>(dq);
+    const uint32_t k_lo = static_cast<uint32_t>(smem_desc_sw128(smem_u32(sKV), 16, 1024));
+    const uint32_t v_lo =
+        static_cast<uint32_t>(smem_desc_sw128(smem_u32(sKV), C::kBoxBytes, 1024));
+    uint32_t L = 0;
+    int qi[NQT] = {0, 0};
+    uint32_t pw[NQT] = {0, 0};
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int idx = item_index(r, cta, G);
+      if (idx >= p.total) break;
+      const Item it = decode_item<CAUSAL>(idx, p, nkv_all);
+      const int nmax = max(it.n0, it.n1);
+      for (int j = 0; ok && j <= nmax; ++j) {
+        const uint32_t Lk = L + 2 * j;
+        const uint32_t Lv = L + 2 * j - 1;
+        bool have_k = false, have_v = false;
 #pragma unroll
-          for (int t = 0; t < NQT; ++t) {
-            if (!ok) break;
-            const int n = t ? it.n1 : it.n0;
-            if (j >= 1 && j - 1 < n) {
-              // O_t (+)= P_t(j-1) V_{j-1}. The p_ready arrival for an item's
-              // first step comes after the softmax group read O_t of its
-              // previous item, so O_t is free to be overwritten here.
-              if (!have_v) {
-                if (!(ok = wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull))) break;
-                have_v = true;
-              }
-              if (!(ok = wait_bar(&p_ready[t], pw[t] & 1, ctl, kSitePReady))) break;
-              ++pw[t];
-              tc_fence_after();
-              const uint32_t vbase = skv + (Lv % S) * C::kTileBytes;
-              const uint32_t tP = tmem + t * BN + kPCol;
-              const uint32_t tO = tmem + C::kOCol + t * D;
-#pragma unroll
-              for (int kk = 0; kk < BN / 16; ++kk) {
-                const uint64_t bdesc =
-                    smem_desc_sw128(vbase + kk * 16 * 128, C::kBoxBytes, 1024);
-                umma_ts(tO, tP + kk * 8, bdesc, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
-              }
-              if (j - 1 == n - 1) umma_commit(&o_done[t]);
+        for (int t = 0; t < NQT; ++t) {
+          if (!ok) break;
+          const int n = t ? it.n1 : it.n0;
+          if (j >= 1 && j - 1 < n) {
+            // O_t (+)= P_t(j-1) V_{j-1}. The p_ready arrival for an item's
+            // first step comes after the softmax group read O_t of its
+            // previous item, so O_t is free to be overwritten here.
+            if (!have_v) {
+              if (!(ok = warp_all(wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull))))
+                break;
+              have_v = true;
             }
-            if (j < n) {
-              // S_t = Q_t K_j^T
-              if (!have_k) {
-                if (!(ok = wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull))) break;
-                tc_fence_after();
-                have_k = true;
-              }
-              if (j == 0) {
-                if (!(ok = wait_bar(&q_full[t], qi[t] & 1, ctl, kSiteQFull))) break;
-                tc_fence_after();
-              }
-              const uint32_t kbase = skv + (Lk % S) * C::kTileBytes;
-              const uint32_t qbase = sq + t * C::kTileBytes;
-              const uint32_t tS = tmem + t * BN;
+            if (!(ok = warp_all(wait_bar(&p_ready[t], pw[t] & 1, ctl, kSitePReady)))) break;
+            ++pw[t];
+            tc_fence_after();
+            const uint32_t vd = v_lo + (((Lv % S) * C::kTileBytes) >> 4);
+            const uint32_t tP = tmem + t * BN + kPCol;
+            const uint32_t tO = tmem + C::kOCol + t * D;
+            // 16 keys = 16 rows of 128 bytes (2048 bytes = 128 in the address field)
+            if (j == 1)
+              umma_ts_w<0>(tO, tP, desc_words(vd, d_hi), idesc_pv);
+            else
+              umma_ts_w<1>(tO, tP, desc_words(vd, d_hi), idesc_pv);
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-                umma_ss(tS, smem_desc_sw128(qbase + koff, 16, 1024),
-                        smem_desc_sw128(kbase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-              }
-              umma_commit(&s_ready[t]);
-              if (j == n - 1) umma_commit(&q_empty[t]);
-            }
+            for (int kk = 1; kk < BN / 16; ++kk)
+              umma_ts_w<1>(tO, tP + kk * 8, desc_words(vd + kk * 128, d_hi), idesc_pv);
+            if (j - 1 == n - 1) umma_commit_w(&o_done[t]);
           }
-          if (have_k) umma_commit(&kv_empty[Lk % S]);
-          if (have_v) umma_commit(&kv_empty[Lv % S]);
+          if (j < n) {
+            // S_t = Q_t K_j^T
+            if (!have_k) {
+              if (!(ok = warp_all(wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull))))
+                break;
+              tc_fence_after();
+              have_k = true;
+            }
+            if (j == 0) {
+              if (!(ok = warp_all(wait_bar(&q_full[t], qi[t] & 1, ctl, kSiteQFull)))) break;
+              tc_fence_after();
+            }
+            const uint32_t kd = k_lo + (((Lk % S) * C::kTileBytes) >> 4);
+            const uint32_t qd = q_lo + ((t * C::kTileBytes) >> 4);
+            const uint32_t tS = tmem + t * BN;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t koff = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+              if (kk == 0)
+                umma_ss_w<0>(tS, desc_words(qd + koff, d_hi), desc_words(kd + koff, d_hi), idesc_s);
+              else
+                umma_ss_w<1>(tS, desc_words(qd + koff, d_hi), desc_words(kd + koff, d_hi), idesc_s);
+            }
+            umma_commit_w(&s_ready[t]);
+            if (j == n - 1) umma_commit_w(&q_empty[t]);
+          }
         }
-        L += 2 * nmax;
-        qi[0] += it.n0 > 0;
-        qi[1] += it.n1 > 0;
+        if (have_k) umma_commit_w(&kv_empty[Lk % S]);
+        if (have_v) umma_commit_w(&kv_empty[Lv % S]);
       }
-      // Every MMA must be complete before tensor memory is released.
-      umma_commit(drain);
-      drain_bar(drain, 0, ctl, kSiteDrain);
+      L += 2 * nmax;
+      qi[0] += it.n0 > 0;
+      qi[1] += it.n1 > 0;
     }
+    // Every MMA must be complete before tensor memory is released.
+    umma_commit_w(drain);
+    drain_bar(drain, 0, ctl, kSiteDrain);
   } else {
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;
