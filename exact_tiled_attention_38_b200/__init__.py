@@ -36,6 +36,8 @@ SIGNATURES = {
     "attn_decode_num_splits": (_I, [_I, _I, _I, _I]),
     "attn_strerror": (ctypes.c_char_p, [_I]),
     "attn_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
+    "attn_fwd_stall_test": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I,
+                                 ctypes.c_uint, _P]),
 }
 
 _lib = None

@@ -351,6 +351,15 @@ int attn_get_device_status(attn_stream_t stream, unsigned int* raw_code) {
   return v == 0 ? ATTN_OK : ATTN_ERR_TIMEOUT;
 }
 
+int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                        unsigned int wait_us, attn_stream_t stream) {
+  if (wait_us < 1 || wait_us > 1000000) return ATTN_ERR_INVALID;
+  return eta::api::fwd<__nv_bfloat16>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                                      reinterpret_cast<cudaStream_t>(stream),
+                                      static_cast<uint64_t>(wait_us) * 1000ull, 1);
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

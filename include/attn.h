@@ -152,6 +152,22 @@ const char* attn_strerror(int code);
  */
 int attn_get_device_status(attn_stream_t stream, unsigned int* raw_code);
 
+/*
+ * Test hook for the bounded waits (not part of the attention computation).
+ * Enqueues the attn_fwd prefill kernel with the same arguments and checks,
+ * but with its TMA producers issuing no copies, so the kernel's first waits
+ * for data can never complete; every wait gives up after wait_us
+ * microseconds (1..1000000). The kernel then ends early with no copy or
+ * tensor-core operation in flight, o and lse are left undefined, and the next
+ * attn_get_device_status() returns ATTN_ERR_TIMEOUT with raw code
+ * 0x1000 | site (site: which wait gave up first). The CUDA context stays
+ * usable. Returns the enqueue status like attn_fwd, or ATTN_ERR_INVALID for
+ * wait_us out of range.
+ */
+int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                        unsigned int wait_us, attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

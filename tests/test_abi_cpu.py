@@ -117,3 +117,10 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(eta, "_lib", None)
     with pytest.raises(RuntimeError):
         eta.load_library(str(tmp_path / "missing.so"))
+
+
+def test_stall_hook_rejects_bad_wait(clib):
+    # checked on the host before any CUDA call
+    for bad in (0, 1000001):
+        assert clib.attn_fwd_stall_test(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 1, 8, 8, 128, 0.1, 1,
+                                        bad, None) == eta.ATTN_ERR_INVALID
