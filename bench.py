@@ -536,6 +536,94 @@ def run_profile(args, local):
     return 0
 
 
+def variant_workloads():
+    """Extra shapes measured by --variants: the long-context prefill configs and
+    the other head groupings, head sizes and dtypes of the same two kernels."""
+    P, D, sb = workloads.PrefillWorkload, workloads.DecodeWorkload, workloads.SEED_BASE + 20
+    return [
+        workloads.PREFILL_GQA_32K,
+        workloads.PREFILL_GQA_128K,
+        P("prefill_noncausal_mha_b4_h16_n4096_d128", 4, 16, 16, 4096, 4096, 128, "bf16", False, sb),
+        P("prefill_causal_mha_b4_h16_n2048_d64", 4, 16, 16, 2048, 2048, 64, "bf16", True, sb + 1),
+        P("prefill_causal_mha_b4_h16_n2048_d128_f16", 4, 16, 16, 2048, 2048, 128, "f16", True,
+          sb + 2),
+        P("prefill_causal_mqa_b2_h32kv1_n4096_d128", 2, 32, 1, 4096, 4096, 128, "bf16", True,
+          sb + 3),
+        P("prefill_chunk_gqa_b1_h32kv8_nq2048_nk32768_d128", 1, 32, 8, 2048, 32768, 128, "bf16",
+          True, sb + 4),
+        D("decode_mqa_b64_h32kv1_d128_ragged", 64, 32, 1, 128, 1024, 8192, "bf16", sb + 5),
+        D("decode_gqa8_b64_h64kv8_d128_ragged", 64, 64, 8, 128, 1024, 8192, "bf16", sb + 6),
+        D("decode_mha_b64_h8kv8_d128_ragged", 64, 8, 8, 128, 1024, 8192, "bf16", sb + 7),
+        D("decode_gqa_b64_h32kv8_d128_ragged_f16", 64, 32, 8, 128, 1024, 8192, "f16", sb + 8),
+        D("decode_gqa_b64_h32kv8_d64_ragged", 64, 32, 8, 64, 1024, 8192, "bf16", sb + 9),
+    ]
+
+
+def run_variants(args, local):
+    """One JSON line per extra workload: median CUDA-event time of single
+    launches, L2 flushed before each, against the measured peaks."""
+    import torch
+
+    import exact_tiled_attention_38_b200 as eta
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    eta.load_library()
+    peaks, _ = load_peaks()
+    flush = torch.empty(64 << 20, dtype=torch.int32, device=dev)
+    flush_rd = torch.empty(64 << 20, dtype=torch.int32, device=dev)
+    for w in variant_workloads():
+        f16 = w.dtype == "f16"
+        if isinstance(w, workloads.PrefillWorkload):
+            q, k, v = workloads.prefill_inputs(w, device=dev)
+            o = torch.empty_like(q)
+            lse = torch.empty(w.B, w.Hq, w.Nq, device=dev, dtype=torch.float32)
+            fn = eta.attn_fwd_f16 if f16 else eta.attn_fwd
+
+            def call():
+                fn(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal)
+
+            work, unit, peak = prefill_flops(w), "TFLOP/s", peaks["bf16_tflops"]
+            scale_units = 1e9
+        else:
+            q, kc, vc, sl = workloads.decode_inputs(w, device=dev)
+            o = torch.empty_like(q)
+            lse = torch.empty(w.B, w.Hq, device=dev, dtype=torch.float32)
+            fn = eta.attn_decode_f16 if f16 else eta.attn_decode
+
+            def call():
+                fn(q, kc, vc, sl, w.Hkv, o=o, lse=lse, scale=w.scale)
+
+            work, unit, peak = decode_kv_bytes(sl.cpu(), w.Hkv, w.d), "GB/s", peaks["hbm_gbs"]
+            scale_units = 1e6
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        reps = 5 if work > 5e13 else 15
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            flush_rd.max()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        code, raw = eta.attn_get_device_status()
+        if code != eta.ATTN_OK:
+            raise RuntimeError(f"{w.name}: device status {code} ({raw:#x})")
+        ms = statistics.median(ts)
+        val = work / ms / scale_units
+        print(json.dumps({"variant": w.name, "value": round(val, 1), "unit": unit,
+                          "ms_per_launch": round(ms, 4), "frac": round(val / peak, 4),
+                          "peak": peak, "launches": reps}), flush=True)
+        del q, o, lse
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -545,6 +633,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=("prefill", "prefill_32k", "decode"), default=None,
                     help="only launch this phase (an ncu target); prints nothing")
+    ap.add_argument("--variants", action="store_true",
+                    help="measure the extra shapes (long context, head groupings, d, dtype), "
+                         "one JSON line each, instead of the step")
     args = ap.parse_args(argv)
     if args.warmup < 3 and not args.profile:
         ap.error("--warmup must be >= 3")
@@ -553,6 +644,8 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.profile:
         return run_profile(args, local)
+    if args.variants:
+        return run_variants(args, local)
     return run_ours(args, world, rank, local)
 
 

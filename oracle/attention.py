@@ -27,7 +27,12 @@ design notes):
   * causal masking is bottom-right aligned: query i sees keys j <= i + Nk - Nq;
   * a row with no visible key has O = 0 and LSE = -inf;
   * the decode cache is packed per sequence as [Hkv][L_b][d] starting at token
-    offset sum(L_0..L_{b-1}); decode attends to all L_b cached tokens.
+    offset sum(L_0..L_{b-1}); decode attends to all L_b cached tokens;
+  * a sliding window of W keys (the "windowing" scheme the zimaspace page names
+    in "Reduced IO Is Not the Same as Eliminating KV Cache") keeps, for causal
+    query i, only keys j with i + Nk - Nq - W < j <= i + Nk - Nq, the W most
+    recent positions including its own; decode with a window reads the last W
+    cached tokens. W = 0 means no window.
 
 ``online_softmax_attention`` and ``combine_partials`` are the method's own
 steps (the running-statistics softmax of "Online Softmax" on the aikaboom page
@@ -63,12 +68,19 @@ def _f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def _visible(nq: int, nk: int, causal: bool, rows: np.ndarray) -> np.ndarray:
-    """Boolean [len(rows), nk]: key j visible to query row i (bottom-right causal)."""
+def _visible(nq: int, nk: int, causal: bool, rows: np.ndarray, window: int = 0) -> np.ndarray:
+    """Boolean [len(rows), nk]: key j visible to query row i (bottom-right causal,
+    optionally limited to the `window` most recent keys)."""
     cols = np.arange(nk)[None, :]
     if not causal:
+        if window:
+            raise ValueError("a sliding window needs the causal mask")
         return np.ones((rows.size, nk), dtype=bool)
-    return cols <= (rows[:, None] + (nk - nq))
+    last = rows[:, None] + (nk - nq)
+    vis = cols <= last
+    if window:
+        vis &= cols > last - window
+    return vis
 
 
 def scores(q_rows: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
@@ -76,13 +88,13 @@ def scores(q_rows: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
     return scale * (q_rows @ k.T)
 
 
-def probabilities(q, k, scale: float, causal: bool) -> np.ndarray:
+def probabilities(q, k, scale: float, causal: bool, window: int = 0) -> np.ndarray:
     """Softmax matrix P for single-head inputs q [Nq, d], k [Nk, d] (two-pass)."""
     q = _f64(q)
     k = _f64(k)
     nq, nk = q.shape[0], k.shape[0]
     s = scores(q, k, scale)
-    s = np.where(_visible(nq, nk, causal, np.arange(nq)), s, -np.inf)
+    s = np.where(_visible(nq, nk, causal, np.arange(nq), window), s, -np.inf)
     m = s.max(axis=1, keepdims=True)
     m_safe = np.where(np.isfinite(m), m, 0.0)
     e = np.exp(s - m_safe)
@@ -93,11 +105,11 @@ def probabilities(q, k, scale: float, causal: bool) -> np.ndarray:
 
 
 def _head_ref(qh: np.ndarray, kh: np.ndarray, vh: np.ndarray, scale: float,
-              causal: bool, nq: int, rows: np.ndarray):
+              causal: bool, nq: int, rows: np.ndarray, window: int = 0):
     """Two-pass attention for one (batch, head) on the given query rows."""
     nk = kh.shape[0]
     s = scores(qh, kh, scale)                       # [R, Nk]
-    s = np.where(_visible(nq, nk, causal, rows), s, -np.inf)
+    s = np.where(_visible(nq, nk, causal, rows, window), s, -np.inf)
     m = s.max(axis=1)                               # pass 1: row max
     m_safe = np.where(np.isfinite(m), m, 0.0)
     e = np.exp(s - m_safe[:, None])                 # pass 2: exponentials
@@ -111,7 +123,7 @@ def _head_ref(qh: np.ndarray, kh: np.ndarray, vh: np.ndarray, scale: float,
     return o, lse
 
 
-def attention_ref(q, k, v, scale: float, causal: bool, rows=None, nq=None):
+def attention_ref(q, k, v, scale: float, causal: bool, rows=None, nq=None, window: int = 0):
     """Exact attention in fp64.
 
     q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] (any float dtype; converted exactly).
@@ -119,6 +131,7 @@ def attention_ref(q, k, v, scale: float, causal: bool, rows=None, nq=None):
     head, or an integer array [B, Hq, R] of per-head rows.
     nq: when given, q holds only the query rows listed in the 1-D ``rows`` (in
     that order) and nq is the full query length the causal mask refers to.
+    window: 0, or the number of most recent keys a causal row sees.
     Returns (O [B, Hq, R, d], LSE [B, Hq, R]) in float64; R = Nq when rows is None.
     """
     q = _f64(q)
@@ -141,7 +154,7 @@ def attention_ref(q, k, v, scale: float, causal: bool, rows=None, nq=None):
             for h in range(Hq):
                 g = h // group
                 out[b, h], lse[b, h] = _head_ref(q[b, h], k[b, g], v[b, g], scale, causal,
-                                                 nq, rows_arr)
+                                                 nq, rows_arr, window)
         return out, lse
     if rows is None:
         rows_arr = np.broadcast_to(np.arange(Nq), (B, Hq, Nq))
@@ -157,7 +170,7 @@ def attention_ref(q, k, v, scale: float, causal: bool, rows=None, nq=None):
             g = h // group
             r = rows_arr[b, h]
             out[b, h], lse[b, h] = _head_ref(q[b, h, r], k[b, g], v[b, g], scale,
-                                             causal, Nq, r)
+                                             causal, Nq, r, window)
     return out, lse
 
 
@@ -190,7 +203,7 @@ def unpack_decode_cache(cache, seqlens, Hkv: int, d: int):
             for o, L in _sequence_ranges(seqlens, Hkv, d)]
 
 
-def decode_ref(q, kcache, vcache, seqlens, scale: float, Hkv: int):
+def decode_ref(q, kcache, vcache, seqlens, scale: float, Hkv: int, window: int = 0):
     """One-token decode over a ragged packed cache, in fp64.
 
     q: [B, Hq, d]; caches packed as described in the module docstring;
@@ -198,6 +211,7 @@ def decode_ref(q, kcache, vcache, seqlens, scale: float, Hkv: int):
     Each new token reads the whole cache of its sequence (the "token generation"
     case on the first page: linear in the number of cached entries).
     Sequences are converted to fp64 one at a time, so large caches fit in memory.
+    window: 0, or the number of most recent cached tokens the new token reads.
     """
     q = _f64(q)
     B, Hq, d = q.shape
@@ -211,13 +225,15 @@ def decode_ref(q, kcache, vcache, seqlens, scale: float, Hkv: int):
             continue
         kb = _f64(kf[o0:o0 + L * Hkv * d]).reshape(1, Hkv, L, d)
         vb = _f64(vf[o0:o0 + L * Hkv * d]).reshape(1, Hkv, L, d)
+        if window:
+            kb, vb = kb[:, :, max(0, L - window):], vb[:, :, max(0, L - window):]
         o, l = attention_ref(q[b][None, :, None, :], kb, vb, scale, causal=False)
         out[b] = o[0, :, 0]
         lse[b] = l[0, :, 0]
     return out, lse
 
 
-def online_softmax_attention(q, k, v, scale: float, causal: bool, tile: int):
+def online_softmax_attention(q, k, v, scale: float, causal: bool, tile: int, window: int = 0):
     """The tiled running-softmax recurrence, for single-head q [Nq,d], k/v [Nk,d].
 
     Key tiles of width ``tile`` are consumed left to right; per query row a
@@ -237,7 +253,7 @@ def online_softmax_attention(q, k, v, scale: float, causal: bool, tile: int):
     for j0 in range(0, nk, tile):
         j1 = min(nk, j0 + tile)
         s = scale * (q @ k[j0:j1].T)
-        vis = _visible(nq, nk, causal, rows)[:, j0:j1]
+        vis = _visible(nq, nk, causal, rows, window)[:, j0:j1]
         s = np.where(vis, s, -np.inf)
         m_new = np.maximum(m, s.max(axis=1))
         m_safe = np.where(np.isfinite(m_new), m_new, 0.0)

@@ -32,6 +32,7 @@ import torch.nn.functional as F
 from torch.nn.attention.bias import causal_lower_right
 
 import oracle
+import workloads
 from oracle import attention as oracle_mod
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -353,7 +354,7 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     good_scores = oracle_mod.scores
     good_head = oracle_mod._head_ref
 
-    def top_left(nq, nk, causal, rows):  # causal aligned top-left instead
+    def top_left(nq, nk, causal, rows, window=0):  # causal aligned top-left instead
         cols = np.arange(nk)[None, :]
         if not causal:
             return np.ones((rows.size, nk), dtype=bool)
@@ -365,8 +366,8 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     def transposed(q_rows, k, scale):
         return scale * (q_rows @ k[::-1].T)
 
-    def lse_without_max(qh, kh, vh, scale, causal, nq, rows):
-        o, lse = good_head(qh, kh, vh, scale, causal, nq, rows)
+    def lse_without_max(qh, kh, vh, scale, causal, nq, rows, window=0):
+        o, lse = good_head(qh, kh, vh, scale, causal, nq, rows, window)
         s = scale * (qh @ kh.T)
         return o, lse - s.max(axis=1)
 
@@ -406,3 +407,127 @@ def test_subset_query_rows_with_full_length():
     o, lse = oracle.attention_ref(q, k, v, 0.4, True, rows=rows)
     o2, lse2 = oracle.attention_ref(q[:, :, rows], k, v, 0.4, True, rows=rows, nq=30)
     assert np.abs(o - o2).max() == 0.0 and np.abs(lse - lse2).max() == 0.0
+
+
+# ------------------------------------------------------------------ sliding window
+# Reading: causal query i keeps keys j with i + off - W < j <= i + off
+# (off = Nk - Nq), the W most recent positions including its own; decode keeps
+# the last W cached tokens (zimaspace page, "Reduced IO Is Not the Same as
+# Eliminating KV Cache", names windowing as a runtime scheme).
+
+def _window_brute(q, k, v, scale, W):
+    """Pure-Python loops over the visible keys of each row (small inputs)."""
+    q, k, v = (oracle_mod._f64(x) for x in (q, k, v))
+    nq, nk, d = q.shape[0], k.shape[0], v.shape[1]
+    off = nk - nq
+    o = np.zeros((nq, d))
+    lse = np.full(nq, -np.inf)
+    for i in range(nq):
+        js = [j for j in range(nk) if i + off - W < j <= i + off]
+        if not js:
+            continue
+        s = [scale * sum(q[i, c] * k[j, c] for c in range(q.shape[1])) for j in js]
+        mx = max(s)
+        e = [math.exp(x - mx) for x in s]
+        tot = sum(e)
+        for jj, j in enumerate(js):
+            o[i] += e[jj] / tot * v[j]
+        lse[i] = mx + math.log(tot)
+    return o, lse
+
+
+@pytest.mark.parametrize("nq,nk,W", [(7, 7, 3), (5, 9, 2), (9, 5, 4), (6, 6, 1), (4, 10, 20)])
+def test_window_matches_brute_force(nq, nk, W):
+    q = _rand((1, 1, nq, 5), 300 + nq)
+    k = _rand((1, 1, nk, 5), 310 + nk)
+    v = _rand((1, 1, nk, 5), 320 + W)
+    o, lse = oracle.attention_ref(q, k, v, 0.7, True, window=W)
+    ob, lb = _window_brute(q[0, 0], k[0, 0], v[0, 0], 0.7, W)
+    fin = np.isfinite(lb)
+    assert np.abs(o[0, 0] - ob).max() < 1e-12
+    assert np.array_equal(np.isfinite(lse[0, 0]), fin)
+    assert np.abs(lse[0, 0][fin] - lb[fin]).max() < 1e-12
+
+
+def test_window_one_key_returns_that_value():
+    q = _rand((1, 2, 6, 4), 330)
+    k = _rand((1, 1, 9, 4), 331)
+    v = _rand((1, 1, 9, 4), 332)
+    o, lse = oracle.attention_ref(q, k, v, 0.5, True, window=1)
+    qq, kk, vv = (oracle_mod._f64(x) for x in (q, k, v))
+    off = 9 - 6
+    for h in range(2):
+        for i in range(6):
+            assert np.array_equal(o[0, h, i], vv[0, 0, i + off])
+            assert abs(lse[0, h, i] - 0.5 * qq[0, h, i] @ kk[0, 0, i + off]) < 1e-12
+
+
+def test_window_wider_than_keys_is_plain_causal():
+    q = _rand((2, 2, 11, 6), 340)
+    k = _rand((2, 1, 11, 6), 341)
+    v = _rand((2, 1, 11, 6), 342)
+    o, lse = oracle.attention_ref(q, k, v, 0.3, True, window=11)
+    o2, lse2 = oracle.attention_ref(q, k, v, 0.3, True)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+
+
+def test_window_ignores_keys_outside_it():
+    q = _rand((1, 1, 8, 4), 350)
+    k = _rand((1, 1, 8, 4), 351)
+    v = _rand((1, 1, 8, 4), 352)
+    o, _ = oracle.attention_ref(q, k, v, 0.6, True, window=3)
+    k2, v2 = k.clone(), v.clone()
+    k2[0, 0, :4] += 5.0  # keys 0..3 are outside the windows of rows 6 and 7
+    v2[0, 0, :4] -= 3.0
+    o2, _ = oracle.attention_ref(q, k2, v2, 0.6, True, window=3)
+    assert np.array_equal(o[0, 0, 6:], o2[0, 0, 6:])
+    assert not np.array_equal(o[0, 0, :4], o2[0, 0, :4])
+
+
+def test_window_online_recurrence_matches_two_pass():
+    q = _rand((1, 1, 13, 6), 360)
+    k = _rand((1, 1, 13, 6), 361)
+    v = _rand((1, 1, 13, 6), 362)
+    o, lse = oracle.attention_ref(q, k, v, 0.4, True, window=5)
+    for tile in (1, 2, 3, 4, 13):
+        ot, lt = oracle.online_softmax_attention(q[0, 0], k[0, 0], v[0, 0], 0.4, True, tile,
+                                                 window=5)
+        assert np.abs(ot - o[0, 0]).max() < 1e-12 and np.abs(lt - lse[0, 0]).max() < 1e-12
+
+
+def test_decode_window_equals_single_row_prefill():
+    # decode reading the last W tokens == causal prefill of one row (Nq = 1) with window W
+    sl = torch.tensor([9, 3, 0, 12], dtype=torch.int32)
+    q, kc, vc, sl = workloads.random_decode(4, 4, 2, 8, sl, torch.float32, seed=370)
+    W = 4
+    o, lse = oracle.decode_ref(q, kc, vc, sl, 0.5, 2, window=W)
+    caches = oracle.unpack_decode_cache(kc, sl, 2, 8), oracle.unpack_decode_cache(vc, sl, 2, 8)
+    for b in range(4):
+        L = int(sl[b])
+        if L == 0:
+            assert np.all(o[b] == 0) and np.all(np.isneginf(lse[b]))
+            continue
+        kb = caches[0][b][None]
+        vb = caches[1][b][None]
+        ob, lb = oracle.attention_ref(q[b][None, :, None, :], kb, vb, 0.5, True, window=W)
+        assert np.abs(ob[0, :, 0] - o[b]).max() < 1e-12
+        assert np.abs(lb[0, :, 0] - lse[b]).max() < 1e-12
+
+
+def test_window_requires_causal():
+    q = _rand((1, 1, 4, 4), 380)
+    with pytest.raises(ValueError):
+        oracle.attention_ref(q, q, q, 0.5, False, window=2)
+
+
+def test_window_pins_catch_an_off_by_one(monkeypatch):
+    good = oracle_mod._visible
+
+    def wide(nq, nk, causal, rows, window=0):  # keeps W + 1 keys
+        return good(nq, nk, causal, rows, window + 1 if window else 0)
+
+    monkeypatch.setattr(oracle_mod, "_visible", wide)
+    with pytest.raises(AssertionError):
+        test_window_matches_brute_force(7, 7, 3)
+    with pytest.raises(AssertionError):
+        test_window_one_key_returns_that_value()
