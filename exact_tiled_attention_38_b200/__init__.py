@@ -38,6 +38,10 @@ SIGNATURES = {
     "attn_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "attn_fwd_stall_test": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I,
                                  ctypes.c_uint, _P]),
+    "attn_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_fwd_window_f16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_decode_window": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_decode_window_f16": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
 }
 
 _lib = None
@@ -92,7 +96,7 @@ def _dev(t, name):
         raise ValueError(f"{name} must be contiguous")
 
 
-def _fwd(fname, dtype, q, k, v, o, lse, scale, causal, stream, want_lse):
+def _fwd(fname, dtype, q, k, v, o, lse, scale, causal, stream, want_lse, window=None):
     import torch
 
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -119,7 +123,8 @@ def _fwd(fname, dtype, q, k, v, o, lse, scale, causal, stream, want_lse):
     fn = getattr(load_library(), fname)
     code = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
               lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
-              float(scale), 1 if causal else 0, _stream_handle(stream))
+              float(scale), *((int(window),) if window is not None else (1 if causal else 0,)),
+              _stream_handle(stream))
     _check(code, fname)
     return o, lse
 
@@ -141,7 +146,8 @@ def attn_fwd_f16(q, k, v, o=None, lse=None, scale: Optional[float] = None,
                 want_lse)
 
 
-def _decode(fname, dtype, q, kcache, vcache, seqlens, Hkv, o, lse, scale, stream, want_lse):
+def _decode(fname, dtype, q, kcache, vcache, seqlens, Hkv, o, lse, scale, stream, want_lse,
+            window=None):
     import torch
 
     for t, n in ((q, "q"), (kcache, "kcache"), (vcache, "vcache"), (seqlens, "seqlens")):
@@ -165,9 +171,31 @@ def _decode(fname, dtype, q, kcache, vcache, seqlens, Hkv, o, lse, scale, stream
     fn = getattr(load_library(), fname)
     code = fn(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
               o.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, d,
-              float(scale), _stream_handle(stream))
+              float(scale), *((int(window),) if window is not None else ()),
+              _stream_handle(stream))
     _check(code, fname)
     return o, lse
+
+
+def attn_fwd_window(q, k, v, window: int, o=None, lse=None, scale: Optional[float] = None,
+                    stream=None, want_lse: bool = True) -> Tuple:
+    """Causal prefill with a sliding window of `window` keys, bf16 (fp16 if q is fp16)."""
+    import torch
+
+    name, dt = (("attn_fwd_window_f16", torch.float16) if q.dtype == torch.float16
+                else ("attn_fwd_window", torch.bfloat16))
+    return _fwd(name, dt, q, k, v, o, lse, scale, True, stream, want_lse, window=window)
+
+
+def attn_decode_window(q, kcache, vcache, seqlens, Hkv: int, window: int, o=None, lse=None,
+                       scale: Optional[float] = None, stream=None, want_lse: bool = True):
+    """Decode reading the last `window` cached tokens, bf16 (fp16 if q is fp16)."""
+    import torch
+
+    name, dt = (("attn_decode_window_f16", torch.float16) if q.dtype == torch.float16
+                else ("attn_decode_window", torch.bfloat16))
+    return _decode(name, dt, q, kcache, vcache, seqlens, Hkv, o, lse, scale, stream, want_lse,
+                   window=window)
 
 
 def attn_decode(q, kcache, vcache, seqlens, Hkv: int, o=None, lse=None,

@@ -61,6 +61,36 @@ int device_info(DeviceInfo* out) {
   return ATTN_OK;
 }
 
+// Stream-ordered workspace for attn_decode: a memory pool owned by the library
+// (one per device). Freed blocks stay cached up to kPoolKeepBytes, so a caller
+// that synchronises between calls does not pay for unmapping and re-mapping
+// device memory on every call (the device's default pool releases its free
+// memory at synchronisation points). The caller's own pools are untouched.
+constexpr uint64_t kPoolKeepBytes = 256ull << 20;
+
+int workspace_pool(cudaMemPool_t* out) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64];
+  static bool have[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!have[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    if (cudaMemPoolCreate(&pools[dev], &props) != cudaSuccess) return ATTN_ERR_CUDA;
+    uint64_t keep = kPoolKeepBytes;
+    if (cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep) !=
+        cudaSuccess)
+      return ATTN_ERR_CUDA;
+    have[dev] = true;
+  }
+  *out = pools[dev];
+  return ATTN_OK;
+}
+
 inline bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
@@ -113,10 +143,10 @@ int launch_fill_empty(void* o, float* lse, long long rows, int D, cudaStream_t s
 #define ETA_PREFILL_POLY8 0
 #endif
 
-template <int D, typename T, bool CAUSAL>
+template <int D, typename T, bool CAUSAL, bool WINDOW = false>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& to, const prefill::Params& p, int grid, cudaStream_t st) {
-  auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, ETA_PREFILL_POLY8, false>;
+  auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, WINDOW, ETA_PREFILL_POLY8, false>;
   constexpr int smem = prefill::Cfg<D>::kSmemBytes;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -131,9 +161,10 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 template <typename T>
 int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
         int Nq, int Nk, int d, float scale, int causal, cudaStream_t st, uint64_t wait_ns,
-        int debug_flags) {
+        int debug_flags, int window = 0) {
   if (B < 0 || Nq < 0 || Nk < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale))
     return ATTN_ERR_INVALID;
+  if (window < 0 || (window > 0 && !causal)) return ATTN_ERR_INVALID;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(Nq) > 65535LL * prefill::NQT * prefill::BM) return ATTN_ERR_INVALID;
   if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return ATTN_ERR_INVALID;
@@ -173,7 +204,11 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = wait_ns;
   p.debug_flags = debug_flags;
+  p.window = window;
   const int grid = static_cast<int>(total < info.sm_count ? total : info.sm_count);
+  if (window > 0)
+    return d == 128 ? launch_prefill<128, T, true, true>(tq, tk, tv, to, p, grid, st)
+                    : launch_prefill<64, T, true, true>(tq, tk, tv, to, p, grid, st);
   if (d == 128)
     return causal ? launch_prefill<128, T, true>(tq, tk, tv, to, p, grid, st)
                   : launch_prefill<128, T, false>(tq, tk, tv, to, p, grid, st);
@@ -234,8 +269,10 @@ int decode_launch_all(const decode::DParams& p, void* o, float* lse, cudaStream_
 
 template <typename T>
 int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* o,
-               float* lse, int B, int Hq, int Hkv, int d, float scale, cudaStream_t st) {
-  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale)) return ATTN_ERR_INVALID;
+               float* lse, int B, int Hq, int Hkv, int d, float scale, cudaStream_t st,
+               int window = 0) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale) || window < 0)
+    return ATTN_ERR_INVALID;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * Hq > 0x7fffffffLL / 4) return ATTN_ERR_INVALID;
   if (B == 0) return ATTN_OK;
@@ -261,11 +298,14 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
   p.nsplit = decode_splits(B, Hq, Hkv, d, info.sm_count);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
+  p.window = window;
 
   const size_t rows = static_cast<size_t>(B) * Hq;
   const size_t bytes = static_cast<size_t>(p.nsplit) * rows * (d + 1) * sizeof(float);
   void* ws = nullptr;
-  if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) return ATTN_ERR_CUDA;
+  cudaMemPool_t pool;
+  if (workspace_pool(&pool) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (cudaMallocFromPoolAsync(&ws, bytes, pool, st) != cudaSuccess) return ATTN_ERR_CUDA;
   p.part_o = reinterpret_cast<float*>(ws);
   p.part_lse = p.part_o + static_cast<size_t>(p.nsplit) * rows * d;
   const int rc = d == 128 ? decode_launch_all<128, T>(p, o, lse, st)
@@ -349,6 +389,41 @@ int attn_get_device_status(attn_stream_t stream, unsigned int* raw_code) {
   }
   if (raw_code != nullptr) *raw_code = v;
   return v == 0 ? ATTN_OK : ATTN_ERR_TIMEOUT;
+}
+
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
+                    attn_stream_t stream) {
+  if (window < 1) return ATTN_ERR_INVALID;
+  return eta::api::fwd<__nv_bfloat16>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1,
+                                      reinterpret_cast<cudaStream_t>(stream),
+                                      eta::kDefaultWaitNs, 0, window);
+}
+
+int attn_fwd_window_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
+                        attn_stream_t stream) {
+  if (window < 1) return ATTN_ERR_INVALID;
+  return eta::api::fwd<__half>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1,
+                               reinterpret_cast<cudaStream_t>(stream), eta::kDefaultWaitNs, 0,
+                               window);
+}
+
+int attn_decode_window(const void* q, const void* kcache, const void* vcache,
+                       const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv, int d,
+                       float scale, int window, attn_stream_t stream) {
+  if (window < 1) return ATTN_ERR_INVALID;
+  return eta::api::decode_run<__nv_bfloat16>(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, d,
+                                             scale, reinterpret_cast<cudaStream_t>(stream),
+                                             window);
+}
+
+int attn_decode_window_f16(const void* q, const void* kcache, const void* vcache,
+                           const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                           int d, float scale, int window, attn_stream_t stream) {
+  if (window < 1) return ATTN_ERR_INVALID;
+  return eta::api::decode_run<__half>(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, d, scale,
+                                      reinterpret_cast<cudaStream_t>(stream), window);
 }
 
 int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -441,6 +516,7 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
   p.nsplit = static_cast<int>(fit < static_cast<size_t>(want) ? fit : want);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
+  p.window = 0;
   // Every partial slot is written by the split pass before the combine reads
   // it, so nothing in the scratch has to start at zero.
   p.part_o = scratch;

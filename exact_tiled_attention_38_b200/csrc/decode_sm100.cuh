@@ -88,6 +88,7 @@ struct DParams {
   int nchunk;  // ceil(G / GP)
   float scale_log2;
   uint64_t wait_ns;
+  int window;  // > 0: each new token reads only the last `window` cached tokens
 };
 
 template <typename T>
@@ -169,9 +170,11 @@ __global__ void __launch_bounds__(kThreads) attn_decode_split_kernel(const DPara
   __syncthreads();
   const long long tok_off = misc[0];
   const int L = static_cast<int>(misc[1]);
-  int per = (L + p.nsplit - 1) / p.nsplit;
+  // Keys read: [tw, L), the whole sequence or its last `window` tokens.
+  const int tw = (p.window > 0 && L > p.window) ? L - p.window : 0;
+  int per = (L - tw + p.nsplit - 1) / p.nsplit;
   per = (per + TK - 1) / TK * TK;
-  const int t_begin = min(L, split * per);
+  const int t_begin = min(L, tw + split * per);
   const int t_end = min(L, t_begin + per);
   const int nkeys = t_end - t_begin;
   const int n_iter = (nkeys + TK - 1) / TK;

@@ -115,6 +115,7 @@ struct Params {
   float scale_log2;
   uint64_t wait_ns;
   int debug_flags;  // bit 0: the producer issues no copies (exercises the wait limit)
+  int window;       // causal only: a row keeps its `window` most recent keys (0 = all)
 };
 
 template <typename T>
@@ -184,13 +185,19 @@ __device__ __forceinline__ uint64_t ex2_poly2(float x0, float x1) {
   return f2_make(r0, r1);
 }
 
+// Key tiles are counted from the item's first one, jb: query tile t uses steps
+// [s_t, n_t), i.e. key tiles jb + s_t .. jb + n_t - 1 (s_t = n_t when the tile
+// has no visible key). Without a window jb = s_0 = s_1 = 0.
 struct Item {
   int bh;
   int b;
   int kvh;
   int r0;  // first query row of tile 0 (tile 1 starts at r0 + BM)
-  int n0;  // key tiles for query tile 0
-  int n1;  // key tiles for query tile 1
+  int jb;  // first key tile the item loads
+  int s0;  // first step of query tile 0
+  int s1;  // first step of query tile 1
+  int n0;  // end step of query tile 0
+  int n1;  // end step of query tile 1
 };
 
 // Snake order over the persistent grid: balances items sorted heaviest first.
@@ -209,7 +216,15 @@ __device__ __forceinline__ int key_tiles(int r0, const Params& p, int nkv_all) {
   return static_cast<int>(ntiles < nkv_all ? ntiles : nkv_all);
 }
 
-template <bool CAUSAL>
+// First key tile any row of the tile starting at r0 sees under the window.
+template <bool CAUSAL, bool WINDOW>
+__device__ __forceinline__ int first_key_tile(int r0, const Params& p) {
+  if (!CAUSAL || !WINDOW) return 0;
+  const long long k0 = static_cast<long long>(r0) + p.off - p.window + 1;
+  return k0 <= 0 ? 0 : static_cast<int>(k0 / BN);
+}
+
+template <bool CAUSAL, bool WINDOW = false>
 __device__ __forceinline__ Item decode_item(int idx, const Params& p, int nkv_all) {
   Item it;
   int pair;
@@ -224,8 +239,15 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, int nkv_al
   const int h = it.bh - it.b * p.Hq;
   it.kvh = h / p.group;
   it.r0 = pair * (NQT * BM);
-  it.n0 = key_tiles<CAUSAL>(it.r0, p, nkv_all);
-  it.n1 = key_tiles<CAUSAL>(it.r0 + BM, p, nkv_all);
+  const int hi0 = key_tiles<CAUSAL>(it.r0, p, nkv_all);
+  const int hi1 = key_tiles<CAUSAL>(it.r0 + BM, p, nkv_all);
+  const int lo0 = min(first_key_tile<CAUSAL, WINDOW>(it.r0, p), hi0);
+  const int lo1 = min(first_key_tile<CAUSAL, WINDOW>(it.r0 + BM, p), hi1);
+  it.jb = (hi0 > lo0) ? lo0 : ((hi1 > lo1) ? lo1 : 0);
+  it.s0 = (hi0 > lo0) ? lo0 - it.jb : 0;
+  it.n0 = (hi0 > lo0) ? hi0 - it.jb : 0;
+  it.s1 = (hi1 > lo1) ? lo1 - it.jb : 0;
+  it.n1 = (hi1 > lo1) ? hi1 - it.jb : 0;
   return it;
 }
 
@@ -267,7 +289,7 @@ __device__ __forceinline__ float exp_tile(const float (&s)[BN], float c, float m
   return (a0 + a1) + (b0 + b1);
 }
 
-template <int D, typename T, bool CAUSAL, int POLY8, bool PINGPONG>
+template <int D, typename T, bool CAUSAL, bool WINDOW, int POLY8, bool PINGPONG>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -342,10 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; ok; ++r) {
         const int idx = item_index(r, cta, G);
         if (idx >= p.total) break;
-        const Item it = decode_item<CAUSAL>(idx, p, nkv_all);
+        const Item it = decode_item<CAUSAL, WINDOW>(idx, p, nkv_all);
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
-          if ((t ? it.n1 : it.n0) == 0) continue;
+          if ((t ? it.n1 - it.s1 : it.n0 - it.s0) <= 0) continue;
           if (qn[t] > 0 && !(ok = wait_bar(&q_empty[t], (qn[t] - 1) & 1, ctl, kSiteQEmpty)))
             break;
           mbar_arrive_expect_tx(&q_full[t], C::kTileBytes);
@@ -364,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
           for (int bx = 0; bx < C::kBoxes; ++bx)
             tma_load_3d(sKV + s * C::kTileBytes + bx * C::kBoxBytes, map, &kv_full[s], bx * 64,
-                        (l >> 1) * BN, zkv);
+                        (it.jb + (l >> 1)) * BN, zkv);
         }
       }
       // No copy may still be landing in shared memory when the CTA exits.
@@ -399,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int r = 0; ok; ++r) {
       const int idx = item_index(r, cta, G);
       if (idx >= p.total) break;
-      const Item it = decode_item<CAUSAL>(idx, p, nkv_all);
+      const Item it = decode_item<CAUSAL, WINDOW>(idx, p, nkv_all);
       const int nmax = max(it.n0, it.n1);
       for (int j = 0; ok && j <= nmax; ++j) {
         const uint32_t Lk = L + 2 * j;
@@ -409,7 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < NQT; ++t) {
           if (!ok) break;
           const int n = t ? it.n1 : it.n0;
-          if (j >= 1 && j - 1 < n) {
+          const int s0 = t ? it.s1 : it.s0;  // this tile's first step
+          if (j >= 1 && j - 1 >= s0 && j - 1 < n) {
             // O_t (+)= P_t(j-1) V_{j-1}. The p_ready arrival for an item's
             // first step comes after the softmax group read O_t of its
             // previous item, so O_t is free to be overwritten here.
@@ -425,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tP = tmem + t * BN + kPCol;
             const uint32_t tO = tmem + C::kOCol + t * D;
             // 16 keys = 16 rows of 128 bytes (2048 bytes = 128 in the address field)
-            if (j == 1)
+            if (j - 1 == s0)
               umma_ts_w<0>(tO, tP, desc_words(vd, d_hi), idesc_pv);
             else
               umma_ts_w<1>(tO, tP, desc_words(vd, d_hi), idesc_pv);
@@ -434,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_ts_w<1>(tO, tP + kk * 8, desc_words(vd + kk * 128, d_hi), idesc_pv);
             if (j - 1 == n - 1) umma_commit_w(&o_done[t]);
           }
-          if (j < n) {
+          if (j >= s0 && j < n) {
             // S_t = Q_t K_j^T
             if (!have_k) {
               if (!(ok = warp_all(wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull))))
@@ -442,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_after();
               have_k = true;
             }
-            if (j == 0) {
+            if (j == s0) {
               if (!(ok = warp_all(wait_bar(&q_full[t], qi[t] & 1, ctl, kSiteQFull)))) break;
               tc_fence_after();
             }
@@ -461,12 +484,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (j == n - 1) umma_commit_w(&q_empty[t]);
           }
         }
+        // A loaded tile that neither query tile uses (a gap between the two
+        // tiles' windows; without a window every loaded tile is used) is still
+        // waited for and released, so the ring keeps its order.
+        if (WINDOW && ok && !have_k && j < nmax) {
+          ok = warp_all(wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull));
+          have_k = ok;
+        }
+        if (WINDOW && ok && !have_v && j >= 1) {
+          ok = warp_all(wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull));
+          have_v = ok;
+        }
         if (have_k) umma_commit_w(&kv_empty[Lk % S]);
         if (have_v) umma_commit_w(&kv_empty[Lv % S]);
       }
       L += 2 * nmax;
-      qi[0] += it.n0 > 0;
-      qi[1] += it.n1 > 0;
+      qi[0] += it.n0 > it.s0;
+      qi[1] += it.n1 > it.s1;
     }
     // Every MMA must be complete before tensor memory is released.
     umma_commit_w(drain);
@@ -489,13 +523,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int r = 0; ok; ++r) {
       const int idx = item_index(r, cta, G);
       if (idx >= p.total) break;
-      const Item it = decode_item<CAUSAL>(idx, p, nkv_all);
+      const Item it = decode_item<CAUSAL, WINDOW>(idx, p, nkv_all);
       const int n = t ? it.n1 : it.n0;
+      const int s0 = t ? it.s1 : it.s0;  // this tile's first step
       const int rt = it.r0 + t * BM;
       const int row = rt + q4 * 32 + lane;
       float m = -INFINITY;  // running max of s * c (log2 units)
       float l = 0.f;        // running sum of p
-      for (int i = 0; i < n; ++i) {
+      for (int i = s0; i < n; ++i) {
         if (!(ok = warp_all(wait_bar(&s_ready[t], sw & 1, ctl, kSiteSReady)))) break;
         ++sw;
         tc_fence_after();
@@ -516,12 +551,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           s[64 + k] = __uint_as_float(rc[k]);
           s[96 + k] = __uint_as_float(rd[k]);
         }
-        const int kv0 = i * BN;
+        const int kv0 = (it.jb + i) * BN;
         const bool edge = (CAUSAL && kv0 + BN - 1 > rt + p.off) || (kv0 + BN > p.Nk);
         if (edge) {
           const int last = (CAUSAL ? min(row + p.off, p.Nk - 1) : p.Nk - 1) - kv0;
 #pragma unroll
           for (int k = 0; k < BN; ++k) s[k] = (k > last) ? -INFINITY : s[k];
+        }
+        // Sliding window: keys before row + off - window + 1 are out of reach.
+        const bool wedge = CAUSAL && WINDOW && kv0 < rt + BM + p.off - p.window;
+        if (wedge) {
+          const int first = row + p.off - p.window + 1 - kv0;
+#pragma unroll
+          for (int k = 0; k < BN; ++k) s[k] = (k < first) ? -INFINITY : s[k];
         }
         // four independent chains of 3-input max, 32 columns each
         float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[32], s[33]);
@@ -547,13 +589,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++tk;
         }
         float lsum;
-        if (POLY8 > 0 && !edge)
+        if (POLY8 > 0 && !edge && !wedge)
           lsum = exp_tile<T, POLY8>(s, sl2, m_use, tP);
         else
           lsum = exp_tile<T, 0>(s, sl2, m_use, tP);
         l += lsum;
         if (PINGPONG) mbar_arrive(&turn[t ^ 1]);
-        if (i > 0 && __any_sync(0xffffffffu, need)) {
+        if (i > s0 && __any_sync(0xffffffffu, need)) {
           // O_t was last written by PV_t(i-1), complete before S_t(i) was signalled.
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -580,8 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (PINGPONG) {
         // Keep the turn order in step with the other group: each group takes
         // max(n0, n1) turns per item.
-        const int nturns = max(it.n0, it.n1);
-        for (int i = n; i < nturns; ++i) {
+        const int nturns = max(it.n0 - it.s0, it.n1 - it.s1);
+        for (int i = n - s0; i < nturns; ++i) {
           if (!(ok = warp_all(wait_bar(&turn[t], tk & 1, ctl, kSiteTurn)))) break;
           ++tk;
           mbar_arrive(&turn[t ^ 1]);
@@ -589,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       if (rt >= p.Nq) continue;  // no rows in this tile
-      if (n > 0) {
+      if (n > s0) {
         if (!(ok = warp_all(wait_bar(&o_done[t], od & 1, ctl, kSiteODone)))) break;
         ++od;
         tc_fence_after();
@@ -608,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cc = 0; cc < 2; ++cc) {
           const int c = half * 2 + cc;
           uint32_t o[32];
-          if (n > 0) {
+          if (n > s0) {
             tmem_ld_x32(tO + c * 32, o);
             tmem_wait_ld_x32(o);
           } else {

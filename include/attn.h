@@ -137,6 +137,32 @@ int attn_decode_noalloc(const void* q, const void* kcache, const void* vcache,
                         const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
                         int d, float scale, attn_stream_t stream);
 
+/*
+ * Sliding-window variants (the "windowing" scheme the zimaspace page names in
+ * "Reduced IO Is Not the Same as Eliminating KV Cache", applied as a mask).
+ * attn_fwd_window: causal prefill where query i keeps only keys j with
+ *   i + (Nk - Nq) - window < j <= i + (Nk - Nq), i.e. its `window` most recent
+ *   positions including its own (bottom-right alignment as in attn_fwd).
+ *   Key tiles wholly outside every row's window are never loaded.
+ * attn_decode_window: the new token of sequence b reads only the last
+ *   min(window, L_b) cached tokens (cache layout as in attn_decode).
+ * window must be >= 1 (a window at least as long as the keys gives the plain
+ * causal / full result). Other arguments, layouts, ownership and errors are
+ * those of attn_fwd / attn_decode; the _f16 twins take and write fp16.
+ */
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
+                    attn_stream_t stream);
+int attn_fwd_window_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
+                        attn_stream_t stream);
+int attn_decode_window(const void* q, const void* kcache, const void* vcache,
+                       const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv, int d,
+                       float scale, int window, attn_stream_t stream);
+int attn_decode_window_f16(const void* q, const void* kcache, const void* vcache,
+                           const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                           int d, float scale, int window, attn_stream_t stream);
+
 /* Number of KV splits attn_decode uses for these sizes on the current device
    (>= 1), or a negative error code. */
 int attn_decode_num_splits(int B, int Hq, int Hkv, int d);

@@ -124,3 +124,11 @@ def test_stall_hook_rejects_bad_wait(clib):
     for bad in (0, 1000001):
         assert clib.attn_fwd_stall_test(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 1, 8, 8, 128, 0.1, 1,
                                         bad, None) == eta.ATTN_ERR_INVALID
+
+
+def test_window_entry_points_reject_bad_windows(clib):
+    for bad in (0, -3):
+        assert clib.attn_fwd_window(FAKE, FAKE, FAKE, FAKE, None, 1, 2, 1, 8, 8, 128, 0.1, bad,
+                                    None) == eta.ATTN_ERR_INVALID
+        assert clib.attn_decode_window(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 2, 1, 128, 0.1,
+                                       bad, None) == eta.ATTN_ERR_INVALID
