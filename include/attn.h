@@ -99,8 +99,12 @@ int attn_fwd_f16(const void* q, const void* k, const void* v, void* o, float* ls
  * Sizes: B >= 0 (0: nothing to do), Hq >= 1, Hkv >= 1, Hq % Hkv == 0,
  * d in {64, 128}.
  * Allocates a split-KV scratch of nsplit * B * Hq * (d + 1) * 4 bytes with
- * cudaMallocAsync on `stream` and frees it with cudaFreeAsync on the same
- * stream (stream-ordered; nothing outlives the call's work).
+ * cudaMallocFromPoolAsync on `stream` and frees it with cudaFreeAsync on the
+ * same stream (stream-ordered; no block outlives the call's work). The pool is
+ * the library's own, one per device, created on first use; it keeps up to
+ * 256 MiB of freed blocks cached, so callers that synchronise between calls do
+ * not pay for re-mapping device memory each time. The caller's pools are not
+ * touched.
  */
 int attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
                 void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
