@@ -11,6 +11,7 @@
 
 #include "../../include/attn.h"
 #include "decode_sm100.cuh"
+#include "generic_fwd.cuh"
 #include "prefill_sm100.cuh"
 
 namespace eta {
@@ -97,6 +98,22 @@ inline bool aligned(const void* p, uintptr_t a) {
 
 inline bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 
+// Head sizes: 64 and 128 run on the tensor-core kernels; any other multiple of
+// 8 from 8 to 256 runs on the CUDA-core generic kernel.
+inline bool tensor_core_d(int d) { return d == 64 || d == 128; }
+inline bool generic_d(int d) { return d >= 8 && d <= generic::kMaxD && d % 8 == 0; }
+
+template <typename T>
+int launch_generic(generic::GParams p, int BH, int Nq, cudaStream_t st) {
+  p.BH = BH;
+  const int ny = BH < generic::kGridY ? BH : generic::kGridY;
+  const dim3 grid((Nq + generic::kRows - 1) / generic::kRows, ny,
+                  (BH + generic::kGridY - 1) / generic::kGridY);
+  generic::attn_generic_kernel<T>
+      <<<grid, generic::kThreads, generic::smem_bytes(p.d), st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 // 3-D map over a [Z][rows][D] tensor of 16-bit elements, box 64 x box_rows x 1,
 // 128-byte swizzle, zero fill outside the tensor (loads) / clipping (stores).
 int encode_3d(CUtensorMap* map, const void* base, bool bf16, int D, long long rows, long long Z,
@@ -165,7 +182,7 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   if (B < 0 || Nq < 0 || Nk < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale))
     return ATTN_ERR_INVALID;
   if (window < 0 || (window > 0 && !causal)) return ATTN_ERR_INVALID;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!tensor_core_d(d) && (!generic_d(d) || debug_flags != 0)) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(Nq) > 65535LL * prefill::NQT * prefill::BM) return ATTN_ERR_INVALID;
   if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return ATTN_ERR_INVALID;
   if (B == 0 || Nq == 0) return ATTN_OK;
@@ -178,6 +195,26 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
   if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
   if (Nk == 0) return launch_fill_empty<T>(o, lse, static_cast<long long>(B) * Hq * Nq, d, st);
+  if (!tensor_core_d(d)) {
+    generic::GParams g;
+    g.q = q;
+    g.k = k;
+    g.v = v;
+    g.o = o;
+    g.lse = lse;
+    g.Hq = Hq;
+    g.Hkv = Hkv;
+    g.Nq = Nq;
+    g.Nk = Nk;
+    g.d = d;
+    g.group = Hq / Hkv;
+    g.off = Nk - Nq;
+    g.causal = causal ? 1 : 0;
+    g.window = window;
+    g.scale_log2 = scale * 1.4426950408889634f;
+    g.seqlens = nullptr;
+    return launch_generic<T>(g, B * Hq, Nq, st);
+  }
 
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap tq, tk, tv, to;
@@ -216,6 +253,20 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                 : launch_prefill<64, T, false>(tq, tk, tv, to, p, grid, st);
 }
 
+// Query heads one split CTA serves: the group padded to 4; larger groups are
+// split into chunks of 4 heads, each chunk reading the cache. A tile of 8
+// heads (ETA_DECODE_MAX_GP=8) reads the cache half as often, but its 8 output
+// rows per lane need 216 registers (one resident CTA fewer per SM) and each
+// key batch carries twice the shuffle and FMA work: measured on B200 for
+// B=64, 1024..8192 tokens, d=128, it took 0.674 / 0.435 / 0.627 ms for
+// groups of 8 / 32 (MQA) / 16 against 0.441 / 0.256 / 0.402 ms with 4, and
+// the same 0.248 ms for a group of 4.
+#ifndef ETA_DECODE_MAX_GP
+#define ETA_DECODE_MAX_GP 4
+#endif
+static_assert(ETA_DECODE_MAX_GP == 4 || ETA_DECODE_MAX_GP == 8, "decode group tile");
+inline int decode_group_tile(int G) { return (G <= 4 || ETA_DECODE_MAX_GP == 4) ? 4 : 8; }
+
 // Split-KV count: enough CTAs for about ETA_DECODE_WAVES waves of resident
 // split CTAs (3 resident per SM), at most 64 splits.
 #ifndef ETA_DECODE_WAVES
@@ -224,7 +275,7 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
 int decode_splits(int B, int Hq, int Hkv, int d, int sm_count) {
   (void)d;
   const int G = Hq / Hkv;
-  const int GP = G <= 4 ? 4 : 8;
+  const int GP = decode_group_tile(G);
   const int nchunk = (G + GP - 1) / GP;
   const long long units = static_cast<long long>(B) * Hkv * nchunk;
   const long long resident = 3LL * sm_count;
@@ -261,10 +312,40 @@ int launch_decode_combine(const float* po, const float* pl, void* o, float* lse,
 
 template <int D, typename T>
 int decode_launch_all(const decode::DParams& p, void* o, float* lse, cudaStream_t st) {
-  const int GP = p.G <= 4 ? 4 : 8;
+#if ETA_DECODE_MAX_GP == 8
+  const int GP = decode_group_tile(p.G);
   int rc = GP == 4 ? launch_decode_split<D, 4, T>(p, st) : launch_decode_split<D, 8, T>(p, st);
+#else
+  int rc = launch_decode_split<D, 4, T>(p, st);
+#endif
   if (rc != ATTN_OK) return rc;
   return launch_decode_combine<D, T>(p.part_o, p.part_lse, o, lse, p.B * p.Hq, p.nsplit, st);
+}
+
+// Decode for head sizes other than 64 and 128: the generic kernel in decode
+// mode, one CTA per (sequence, query head), no workspace.
+template <typename T>
+int decode_generic(const void* q, const void* kc, const void* vc, const int32_t* seqlens,
+                   void* o, float* lse, int B, int Hq, int Hkv, int d, float scale, int window,
+                   cudaStream_t st) {
+  generic::GParams g;
+  g.q = q;
+  g.k = kc;
+  g.v = vc;
+  g.o = o;
+  g.lse = lse;
+  g.Hq = Hq;
+  g.Hkv = Hkv;
+  g.Nq = 1;
+  g.Nk = 0;  // per sequence, from seqlens
+  g.d = d;
+  g.group = Hq / Hkv;
+  g.off = 0;
+  g.causal = 1;
+  g.window = window;
+  g.scale_log2 = scale * 1.4426950408889634f;
+  g.seqlens = seqlens;
+  return launch_generic<T>(g, B * Hq, 1, st);
 }
 
 template <typename T>
@@ -273,7 +354,7 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
                int window = 0) {
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale) || window < 0)
     return ATTN_ERR_INVALID;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!tensor_core_d(d) && !generic_d(d)) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * Hq > 0x7fffffffLL / 4) return ATTN_ERR_INVALID;
   if (B == 0) return ATTN_OK;
   if (q == nullptr || kc == nullptr || vc == nullptr || seqlens == nullptr || o == nullptr ||
@@ -283,6 +364,8 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
   DeviceInfo info;
   if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
   if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
+  if (!tensor_core_d(d))
+    return decode_generic<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, window, st);
 
   decode::DParams p;
   p.q = q;
@@ -293,7 +376,7 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
-  const int GP = p.G <= 4 ? 4 : 8;
+  const int GP = decode_group_tile(p.G);
   p.nchunk = (p.G + GP - 1) / GP;
   p.nsplit = decode_splits(B, Hq, Hkv, d, info.sm_count);
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -350,7 +433,7 @@ int attn_decode_f16(const void* q, const void* kcache, const void* vcache,
 
 int attn_decode_num_splits(int B, int Hq, int Hkv, int d) {
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!eta::api::tensor_core_d(d)) return eta::api::generic_d(d) ? 1 : ATTN_ERR_UNSUPPORTED;
   eta::api::DeviceInfo info;
   if (eta::api::device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
   return eta::api::decode_splits(B, Hq, Hkv, d, info.sm_count);
@@ -482,13 +565,19 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
                        void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
                        cudaStream_t st) {
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale)) return ATTN_ERR_INVALID;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!tensor_core_d(d) && !generic_d(d)) return ATTN_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * Hq > 0x7fffffffLL / 4) return ATTN_ERR_INVALID;
   if (B == 0) return ATTN_OK;
   if (q == nullptr || kc == nullptr || vc == nullptr || seqlens == nullptr || o == nullptr ||
       !aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(o, 16) ||
       !aligned(seqlens, 4) || (lse != nullptr && !aligned(lse, 4)))
     return ATTN_ERR_INVALID;
+  if (!tensor_core_d(d)) {  // the generic kernel needs no scratch
+    DeviceInfo info;
+    if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
+    if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
+    return decode_generic<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, 0, st);
+  }
   // One split needs B * Hq * (d + 1) floats; fewer splits are used when the
   // usual count does not fit, and sizes where even one does not fit are refused.
   const size_t rows = static_cast<size_t>(B) * Hq;
@@ -509,7 +598,7 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
-  const int GP = p.G <= 4 ? 4 : 8;
+  const int GP = decode_group_tile(p.G);
   p.nchunk = (p.G + GP - 1) / GP;
   const size_t fit = kNoAllocScratchFloats / per_split;
   const int want = decode_splits(B, Hq, Hkv, d, info.sm_count);

@@ -35,6 +35,12 @@
  *     code before anything is enqueued.
  *   - A row with no visible key (causal with Nq > Nk, or an empty decode
  *     sequence) gets o = 0 and lse = -inf.
+ *   - Head size d: d = 64 and d = 128 run on the tensor-core kernels
+ *     (tcgen05 MMA, TMA-fed tiles). Any other d that is a multiple of 8 in
+ *     [8, 256] runs on a generic CUDA-core kernel with the same results to
+ *     rounding (16 query rows per block, 32-key tiles staged in shared
+ *     memory, fp32 online softmax); it is correct but far from the tensor-core
+ *     kernels' speed. Other d return ATTN_ERR_UNSUPPORTED.
  *   - Every wait inside a kernel is bounded (about 2 s). If one gives up, the
  *     kernel ends early, its outputs are undefined, and
  *     attn_get_device_status() reports ATTN_ERR_TIMEOUT. No kernel traps.
@@ -55,7 +61,7 @@ typedef struct CUstream_st* attn_stream_t;
 enum attn_status {
   ATTN_OK = 0,
   ATTN_ERR_INVALID = -1,     /* null pointer, bad size, misaligned, Hq % Hkv != 0, bad scale */
-  ATTN_ERR_UNSUPPORTED = -2, /* d not in {64, 128}, or the device is not sm_100 */
+  ATTN_ERR_UNSUPPORTED = -2, /* d not a multiple of 8 in [8, 256], or the device is not sm_100 */
   ATTN_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
   ATTN_ERR_TIMEOUT = -4,     /* a device-side wait gave up (see attn_get_device_status) */
   ATTN_ERR_SCRATCH = -5      /* attn_decode_noalloc: sizes exceed its fixed scratch */
@@ -71,7 +77,7 @@ enum attn_status {
  *                (equal to the usual lower-triangular mask when Nq == Nk).
  * Sizes: B >= 0, Nq >= 0, Nk >= 0 (B == 0 or Nq == 0: nothing to do;
  * Nk == 0: every row is empty), Hq >= 1, Hkv >= 1, Hq % Hkv == 0,
- * d in {64, 128}, Nq <= 16,776,960.
+ * d a multiple of 8 in [8, 256], Nq <= 16,776,960 (generic d: B * Hq <= 65,535).
  * Allocates no device memory.
  */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -97,14 +103,15 @@ int attn_fwd_f16(const void* q, const void* k, const void* v, void* o, float* ls
  *           values count as 0; 0 gives o = 0, lse = -inf).
  *   o       [B, Hq, d]  bf16       lse [B, Hq] float32 (or NULL)
  * Sizes: B >= 0 (0: nothing to do), Hq >= 1, Hkv >= 1, Hq % Hkv == 0,
- * d in {64, 128}.
- * Allocates a split-KV scratch of nsplit * B * Hq * (d + 1) * 4 bytes with
+ * d a multiple of 8 in [8, 256] (generic d: B * Hq <= 65,535).
+ * For d = 64 and 128, allocates a split-KV scratch of nsplit * B * Hq * (d + 1) * 4 bytes with
  * cudaMallocFromPoolAsync on `stream` and frees it with cudaFreeAsync on the
  * same stream (stream-ordered; no block outlives the call's work). The pool is
  * the library's own, one per device, created on first use; it keeps up to
  * 256 MiB of freed blocks cached, so callers that synchronise between calls do
  * not pay for re-mapping device memory each time. The caller's pools are not
- * touched.
+ * touched. Other d use one block per (sequence, query head), no split and no
+ * scratch.
  */
 int attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
                 void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
@@ -168,7 +175,7 @@ int attn_decode_window_f16(const void* q, const void* kcache, const void* vcache
                            int d, float scale, int window, attn_stream_t stream);
 
 /* Number of KV splits attn_decode uses for these sizes on the current device
-   (>= 1), or a negative error code. */
+   (>= 1; always 1 for d other than 64 and 128), or a negative error code. */
 int attn_decode_num_splits(int B, int Hq, int Hkv, int d);
 
 /* Human-readable text for a return code. Never NULL. */
@@ -192,7 +199,8 @@ int attn_get_device_status(attn_stream_t stream, unsigned int* raw_code);
  * attn_get_device_status() returns ATTN_ERR_TIMEOUT with raw code
  * 0x1000 | site (site: which wait gave up first). The CUDA context stays
  * usable. Returns the enqueue status like attn_fwd, or ATTN_ERR_INVALID for
- * wait_us out of range.
+ * wait_us out of range, or ATTN_ERR_UNSUPPORTED for d other than 64 and 128
+ * (the generic kernel has no waits).
  */
 int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,

@@ -80,8 +80,12 @@ def test_fwd_host_validation(clib):
     assert fwd(clib, Nq=-5) == eta.ATTN_ERR_INVALID
     assert fwd(clib, scale=0.0) == eta.ATTN_ERR_INVALID
     assert fwd(clib, scale=float("inf")) == eta.ATTN_ERR_INVALID
-    assert fwd(clib, d=96) == eta.ATTN_ERR_UNSUPPORTED
-    assert fwd(clib, d=256) == eta.ATTN_ERR_UNSUPPORTED
+    # head sizes: multiples of 8 in [8, 256] are taken (64 and 128 on the
+    # tensor cores, the rest on the generic kernel); nothing else is
+    for d in (0, 4, 12, 100, 264, 512):
+        assert fwd(clib, d=d) == eta.ATTN_ERR_UNSUPPORTED, d
+    for d in (8, 96, 256):  # accepted: an empty problem is a no-op
+        assert fwd(clib, d=d, B=0) == eta.ATTN_OK, d
     assert fwd(clib, o=None) == eta.ATTN_ERR_INVALID
     assert fwd(clib, q=ctypes.c_void_p(0x10008)) == eta.ATTN_ERR_INVALID
     assert fwd(clib, lse=ctypes.c_void_p(0x10002)) == eta.ATTN_ERR_INVALID
@@ -104,13 +108,16 @@ def dec(clib, **kw):
 def test_decode_host_validation(clib):
     assert dec(clib, Hq=6, Hkv=4) == eta.ATTN_ERR_INVALID
     assert dec(clib, scale=-0.5) == eta.ATTN_ERR_INVALID
-    assert dec(clib, d=80) == eta.ATTN_ERR_UNSUPPORTED
+    assert dec(clib, d=84) == eta.ATTN_ERR_UNSUPPORTED
+    assert dec(clib, d=272) == eta.ATTN_ERR_UNSUPPORTED
+    assert dec(clib, d=80, B=0) == eta.ATTN_OK
     assert dec(clib, s=None) == eta.ATTN_ERR_INVALID
     assert dec(clib, s=ctypes.c_void_p(0x10002)) == eta.ATTN_ERR_INVALID
     assert dec(clib, k=ctypes.c_void_p(0x10004)) == eta.ATTN_ERR_INVALID
     assert dec(clib, B=0) == eta.ATTN_OK
     assert clib.attn_decode_num_splits(2, 6, 4, 128) == eta.ATTN_ERR_INVALID
-    assert clib.attn_decode_num_splits(2, 8, 2, 96) == eta.ATTN_ERR_UNSUPPORTED
+    assert clib.attn_decode_num_splits(2, 8, 2, 100) == eta.ATTN_ERR_UNSUPPORTED
+    assert clib.attn_decode_num_splits(2, 8, 2, 96) == 1  # generic kernel: no split
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
@@ -124,6 +131,9 @@ def test_stall_hook_rejects_bad_wait(clib):
     for bad in (0, 1000001):
         assert clib.attn_fwd_stall_test(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 1, 8, 8, 128, 0.1, 1,
                                         bad, None) == eta.ATTN_ERR_INVALID
+    # the generic head-size kernel has no waits to stall
+    assert clib.attn_fwd_stall_test(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 1, 8, 8, 96, 0.1, 1,
+                                    1000, None) == eta.ATTN_ERR_UNSUPPORTED
 
 
 def test_window_entry_points_reject_bad_windows(clib):

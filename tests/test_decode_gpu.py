@@ -47,6 +47,7 @@ CASES = [
     (2, 8, 8, 128, [0, 0], BF16),              # every sequence empty
     (1, 8, 2, 128, [20000], F16),              # one long sequence over many splits
     (5, 12, 4, 128, [1, 2, 3, 4, 5], BF16),
+    (2, 12, 2, 64, [300, 1000], F16),          # group 6: one full chunk of 4, one of 2
 ]
 
 

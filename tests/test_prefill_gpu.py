@@ -138,7 +138,7 @@ def test_rejects_bad_arguments_on_gpu(lib):
     with pytest.raises(lib.AttnError) as e:
         lib.attn_fwd(mis, q, q)
     assert e.value.code == lib.ATTN_ERR_INVALID
-    q96 = torch.randn(1, 2, 16, 96, device=DEV).to(BF16)
+    q100 = torch.randn(1, 2, 16, 100, device=DEV).to(BF16)
     with pytest.raises(lib.AttnError) as e:
-        lib.attn_fwd(q96, q96, q96)
+        lib.attn_fwd(q100, q100, q100)
     assert e.value.code == lib.ATTN_ERR_UNSUPPORTED
