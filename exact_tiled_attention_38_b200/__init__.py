@@ -42,6 +42,8 @@ SIGNATURES = {
     "attn_fwd_window_f16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_decode_window": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "attn_decode_window_f16": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_merge": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _P]),
+    "attn_merge_f16": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _P]),
 }
 
 _lib = None
@@ -229,6 +231,41 @@ def attn_decode_noalloc(q, kcache, vcache, seqlens, Hkv: int, o=None, lse=None,
 
     return _decode("attn_decode_noalloc", torch.bfloat16, q, kcache, vcache, seqlens, Hkv, o,
                    lse, scale, stream, want_lse)
+
+
+def attn_merge(o_acc, lse_acc, o_part, lse_part, o_out=None, stream=None) -> None:
+    """Fold a partial result (o_part, lse_part) into the fp32 accumulator in place.
+
+    o_acc float32 [..., d] and lse_acc float32 [...] (same leading shape as
+    o_part / lse_part); o_part bf16 or fp16; o_out (optional, o_part's dtype
+    and shape) also receives the merged O rounded. A row with lse_acc = -inf is
+    empty (o_acc not read). Runs ``attn_merge`` / ``attn_merge_f16``.
+    """
+    import torch
+
+    for t, n in ((o_acc, "o_acc"), (lse_acc, "lse_acc"), (o_part, "o_part"),
+                 (lse_part, "lse_part")):
+        _dev(t, n)
+    if o_part.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("o_part must be bf16 or fp16")
+    if o_acc.dtype != torch.float32 or lse_acc.dtype != torch.float32 or \
+            lse_part.dtype != torch.float32:
+        raise ValueError("o_acc, lse_acc and lse_part must be float32")
+    d = o_part.shape[-1]
+    if tuple(o_acc.shape) != tuple(o_part.shape) or \
+            tuple(lse_acc.shape) != tuple(o_part.shape[:-1]) or \
+            tuple(lse_part.shape) != tuple(o_part.shape[:-1]):
+        raise ValueError("o_acc, lse_acc, o_part and lse_part shapes disagree")
+    if o_out is not None:
+        _dev(o_out, "o_out")
+        if o_out.dtype != o_part.dtype or tuple(o_out.shape) != tuple(o_part.shape):
+            raise ValueError("o_out must match o_part")
+    name = "attn_merge_f16" if o_part.dtype == torch.float16 else "attn_merge"
+    rows = o_part.numel() // d if d else 0
+    code = getattr(load_library(), name)(
+        o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+        o_out.data_ptr() if o_out is not None else None, rows, d, _stream_handle(stream))
+    _check(code, name)
 
 
 def attn_decode_num_splits(B: int, Hq: int, Hkv: int, d: int) -> int:

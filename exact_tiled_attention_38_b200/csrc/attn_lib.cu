@@ -12,6 +12,7 @@
 #include "../../include/attn.h"
 #include "decode_sm100.cuh"
 #include "generic_fwd.cuh"
+#include "merge.cuh"
 #include "prefill_sm100.cuh"
 
 namespace eta {
@@ -401,6 +402,36 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
 }  // namespace api
 }  // namespace eta
 
+namespace eta {
+namespace api {
+
+template <typename T>
+int merge_run(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+              void* o_out, long long rows, int d, cudaStream_t st) {
+  if (rows < 0 || !generic_d(d)) return rows < 0 ? ATTN_ERR_INVALID : ATTN_ERR_UNSUPPORTED;
+  if (rows > (0x7fffffffffffLL / d)) return ATTN_ERR_INVALID;
+  if (rows == 0) return ATTN_OK;
+  if (o_acc == nullptr || lse_acc == nullptr || o_part == nullptr || lse_part == nullptr ||
+      !aligned(o_acc, 16) || !aligned(o_part, 16) || !aligned(lse_acc, 4) ||
+      !aligned(lse_part, 4) || (o_out != nullptr && !aligned(o_out, 16)))
+    return ATTN_ERR_INVALID;
+  DeviceInfo info;
+  if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
+  const int rpw = 32 / (d / 8);
+  const long long rows_per_block = static_cast<long long>(rpw) * (merge::kThreads / 32);
+  const long long want = (rows + rows_per_block - 1) / rows_per_block;
+  const long long cap = 8LL * info.sm_count;  // grid-stride beyond 8 blocks per SM
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  merge::attn_merge_kernel<T><<<blocks, merge::kThreads, 0, st>>>(
+      o_acc, lse_acc, reinterpret_cast<const T*>(o_part), lse_part, reinterpret_cast<T*>(o_out),
+      rows, d);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace api
+}  // namespace eta
+
 extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -507,6 +538,18 @@ int attn_decode_window_f16(const void* q, const void* kcache, const void* vcache
   if (window < 1) return ATTN_ERR_INVALID;
   return eta::api::decode_run<__half>(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, d, scale,
                                       reinterpret_cast<cudaStream_t>(stream), window);
+}
+
+int attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+               void* o_out, long long rows, int d, attn_stream_t stream) {
+  return eta::api::merge_run<__nv_bfloat16>(o_acc, lse_acc, o_part, lse_part, o_out, rows, d,
+                                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_merge_f16(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                   void* o_out, long long rows, int d, attn_stream_t stream) {
+  return eta::api::merge_run<__half>(o_acc, lse_acc, o_part, lse_part, o_out, rows, d,
+                                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -174,6 +174,35 @@ int attn_decode_window_f16(const void* q, const void* kcache, const void* vcache
                            const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
                            int d, float scale, int window, attn_stream_t stream);
 
+/*
+ * Merge of partial results over disjoint key sets (context-parallel prefill:
+ * each step computes a query block's attention over one key block with
+ * attn_fwd, and the steps' results are folded together). The log-sum-exp
+ * identity follows from the running softmax statistics (aikaboom page
+ * "11.4d FlashAttention", "Online Softmax"): for one query row,
+ *     LSE = ln(e^lse_acc + e^lse_part)
+ *     O   = e^(lse_acc - LSE) * o_acc + e^(lse_part - LSE) * o_part.
+ *   o_acc    [rows, d] float32, in/out: the running merged O (unrounded)
+ *   lse_acc  [rows]    float32, in/out: the running LSE (natural log). A row
+ *            whose lse_acc is -inf is empty and its o_acc is NOT read, so an
+ *            accumulator starts as lse_acc = -inf with o_acc uninitialised.
+ *   o_part   [rows, d] bf16 (attn_merge) or fp16 (attn_merge_f16), and
+ *   lse_part [rows]    float32: one partial result, e.g. attn_fwd's o and lse
+ *            over a key block (rows = B * Hq * Nq in attn_fwd's layout). A
+ *            partial row with lse_part = -inf (no visible key) changes nothing.
+ *   o_out    [rows, d] bf16 / fp16, or NULL: if not NULL, also receives the
+ *            merged O rounded to nearest (the final merge of a sequence of
+ *            merges writes the output this way); rows that stay empty get 0.
+ * Sizes: rows >= 0 (0: nothing to do), d a multiple of 8 in [8, 256].
+ * Pointers are device pointers owned by the caller; o_acc, o_part and o_out
+ * 16-byte aligned, lse_acc and lse_part 4-byte aligned. o_out must not
+ * overlap the other arrays. Allocates nothing.
+ */
+int attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+               void* o_out, long long rows, int d, attn_stream_t stream);
+int attn_merge_f16(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                   void* o_out, long long rows, int d, attn_stream_t stream);
+
 /* Number of KV splits attn_decode uses for these sizes on the current device
    (>= 1; always 1 for d other than 64 and 128), or a negative error code. */
 int attn_decode_num_splits(int B, int Hq, int Hkv, int d);

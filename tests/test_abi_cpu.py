@@ -142,3 +142,22 @@ def test_window_entry_points_reject_bad_windows(clib):
                                     None) == eta.ATTN_ERR_INVALID
         assert clib.attn_decode_window(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 2, 1, 128, 0.1,
                                        bad, None) == eta.ATTN_ERR_INVALID
+
+
+def test_merge_host_validation(clib):
+    def merge(**kw):
+        a = dict(oa=FAKE, la=FAKE, op=FAKE, lp=FAKE, out=None, rows=10, d=128)
+        a.update(kw)
+        return clib.attn_merge(a["oa"], a["la"], a["op"], a["lp"], a["out"], a["rows"], a["d"],
+                               None)
+
+    assert merge(rows=-1) == eta.ATTN_ERR_INVALID
+    assert merge(d=12) == eta.ATTN_ERR_UNSUPPORTED
+    assert merge(d=264) == eta.ATTN_ERR_UNSUPPORTED
+    assert merge(rows=0) == eta.ATTN_OK
+    assert merge(oa=None) == eta.ATTN_ERR_INVALID
+    assert merge(lp=None) == eta.ATTN_ERR_INVALID
+    assert merge(op=ctypes.c_void_p(0x10008)) == eta.ATTN_ERR_INVALID
+    assert merge(la=ctypes.c_void_p(0x10002)) == eta.ATTN_ERR_INVALID
+    assert merge(out=ctypes.c_void_p(0x10004)) == eta.ATTN_ERR_INVALID
+    assert clib.attn_merge_f16(FAKE, FAKE, FAKE, FAKE, None, 0, 64, None) == eta.ATTN_OK
