@@ -601,7 +601,62 @@ def run_variants(args, local):
         torch.cuda.synchronize()
         reps = 5 if work > 5e13 else 15
         ts = []
-        for _ in range(reps):
+        with ClockSampler(local) as clocks:
+            for _ in range(reps):
+                flush.zero_()
+                flush_rd.max()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                call()
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+        code, raw = eta.attn_get_device_status()
+        if code != eta.ATTN_OK:
+            raise RuntimeError(f"{w.name}: device status {code} ({raw:#x})")
+        ms = statistics.median(ts)
+        val = work / ms / scale_units
+        line = {"variant": w.name, "value": round(val, 1), "unit": unit,
+                "ms_per_launch": round(ms, 4), "frac": round(val / peak, 4), "peak": peak,
+                "launches": reps, "clocks": clocks.summary()}
+        if unit == "TFLOP/s" and "bf16_tflops_sustained" in peaks:
+            line["frac_sustained"] = round(val / peaks["bf16_tflops_sustained"], 4)
+        print(json.dumps(line), flush=True)
+        del q, o, lse
+        torch.cuda.empty_cache()
+    run_ring_variant(eta, dev, local, peaks, flush, flush_rd)
+    return 0
+
+
+def run_ring_variant(eta, dev, local, peaks, flush, flush_rd, world=8):
+    """Context-parallel prefill of the 128K causal GQA workload over an
+    8-rank zigzag ring: rank 0's whole call sequence (8 steps, 2 chunk pairs
+    each, plus the LSE merges) on this one GPU, with LocalRing's device copies
+    standing in for the K/V transfers. Every rank does the same work, so the
+    per-rank rate is what each GPU of an 8-GPU ring would compute."""
+    import torch
+
+    from exact_tiled_attention_38_b200 import context_parallel as cp
+
+    w = workloads.PREFILL_GQA_128K
+    q, k, v = workloads.prefill_inputs(w, device=dev)
+    ks = [cp.shard_zigzag(k, r, world) for r in range(world)]
+    vs = [cp.shard_zigzag(v, r, world) for r in range(world)]
+    q0 = cp.shard_zigzag(q, 0, world)
+    del q, k, v
+    torch.cuda.empty_cache()
+    c = w.Nq // (2 * world)
+    flops = 4.0 * w.d * w.Hq * w.B * (2 * world * c * c + c)  # one rank's visible pairs
+
+    def call():
+        cp.ring_attention(q0, ks[0], vs[0], True, w.scale, exchange=cp.LocalRing(0, ks, vs))
+
+    call()
+    torch.cuda.synchronize()
+    ts = []
+    with ClockSampler(local) as clocks:
+        for _ in range(3):
             flush.zero_()
             flush_rd.max()
             e0 = torch.cuda.Event(enable_timing=True)
@@ -611,17 +666,18 @@ def run_variants(args, local):
             e1.record()
             torch.cuda.synchronize()
             ts.append(e0.elapsed_time(e1))
-        code, raw = eta.attn_get_device_status()
-        if code != eta.ATTN_OK:
-            raise RuntimeError(f"{w.name}: device status {code} ({raw:#x})")
-        ms = statistics.median(ts)
-        val = work / ms / scale_units
-        print(json.dumps({"variant": w.name, "value": round(val, 1), "unit": unit,
-                          "ms_per_launch": round(ms, 4), "frac": round(val / peak, 4),
-                          "peak": peak, "launches": reps}), flush=True)
-        del q, o, lse
-        torch.cuda.empty_cache()
-    return 0
+    code, raw = eta.attn_get_device_status()
+    if code != eta.ATTN_OK:
+        raise RuntimeError(f"ring: device status {code} ({raw:#x})")
+    ms = statistics.median(ts)
+    val = flops / ms / 1e9
+    print(json.dumps({"variant": f"prefill_ring_w{world}_rank0_causal_gqa_b1_h32kv8_n128k_d128",
+                      "value": round(val, 1), "unit": "TFLOP/s", "ms_per_launch": round(ms, 4),
+                      "frac": round(val / peaks["bf16_tflops"], 4), "peak": peaks["bf16_tflops"],
+                      "launches": len(ts), "chunk": c, "clocks": clocks.summary(),
+                      "frac_sustained": round(val / peaks.get("bf16_tflops_sustained",
+                                                              peaks["bf16_tflops"]), 4)}),
+          flush=True)
 
 
 def main(argv=None):
