@@ -373,6 +373,23 @@ def run_ours(args, world, rank, local):
         if evs:
             evs[2].record(stream)
 
+    # Device memory the library itself holds (device-wide free bytes before and
+    # after the first call of each): prefill allocates nothing; decode keeps its
+    # split workspace cached in the library's pool. A materialised fp32 score
+    # matrix would take B * Hq * Nq * Nk * 4 bytes.
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info(dev)[0]
+    eta.attn_fwd(q, k, v, o=o, lse=lse, scale=PREFILL.scale, causal=True, stream=stream)
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info(dev)[0]
+    eta.attn_decode(dq, dkc, dvc, dsl, DECODE.Hkv, o=do, lse=dlse, scale=DECODE.scale,
+                    stream=stream)
+    torch.cuda.synchronize()
+    free2 = torch.cuda.mem_get_info(dev)[0]
+    memory = {"prefill_library_bytes": free0 - free1, "decode_library_bytes": free1 - free2,
+              "prefill_score_matrix_fp32_bytes": PREFILL.B * PREFILL.Hq * PREFILL.Nq *
+              PREFILL.Nk * 4, "how": "device-wide free memory before and after the first call"}
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -471,6 +488,7 @@ def run_ours(args, world, rank, local):
             "l2": "flushed before every step (256 MiB write, then a 256 MiB read that "
                   "evicts its dirty lines; outside the kernel events)",
             "parallelism": f"replicas x{world} (independent batches per GPU)",
+            "memory": memory,
         },
         # The dominant kernel of a step (by the committed launch-list share and
         # by the events here) is the decode split pass; its roofline is the

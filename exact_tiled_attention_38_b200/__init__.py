@@ -42,6 +42,7 @@ SIGNATURES = {
     "attn_fwd_window_f16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_decode_window": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "attn_decode_window_f16": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_last_cuda_error": (_I, []),
     "attn_merge": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _P]),
     "attn_merge_f16": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _P]),
 }
@@ -52,7 +53,9 @@ _lib = None
 class AttnError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {strerror(code)} (code {code})")
+        self.cuda_error = load_library().attn_last_cuda_error() if code == ATTN_ERR_CUDA else 0
+        extra = f", cudaError {self.cuda_error}" if self.cuda_error else ""
+        super().__init__(f"{where}: {strerror(code)} (code {code}{extra})")
 
 
 def load_library(path: str = LIB_PATH):

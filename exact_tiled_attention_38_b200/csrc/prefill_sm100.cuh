@@ -58,9 +58,12 @@ namespace prefill {
 constexpr int BM = 128;   // query rows per tile
 constexpr int BN = 128;   // keys per tile
 constexpr int NQT = 2;    // query tiles per CTA
-constexpr int kThreads = 320;
-constexpr int kMmaWarp = 8;
-constexpr int kTmaWarp = 9;
+// SPLIT softmax threads share a query row (SPLIT = 1: 4 warps per query tile;
+// SPLIT = 2: 8 warps per tile, each thread taking 64 of the row's 128 scores).
+__host__ __device__ constexpr int softmax_warps(int split) { return 4 * NQT * split; }
+__host__ __device__ constexpr int kernel_threads(int split) {
+  return 32 * (softmax_warps(split) + 2);
+}
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kPCol = 64;  // P_t starts this many columns into S_t
@@ -76,6 +79,8 @@ enum : unsigned {
   kSiteDrain = 7,
   kSiteQEmpty = 8,
   kSiteTurn = 9,
+  kSiteXUp = 10,
+  kSiteXDown = 11,
 };
 
 template <int D>
@@ -92,10 +97,14 @@ struct Cfg {
   static constexpr int kStgOff = kKVOff + kStages * kTileBytes;
   static constexpr int kBarOff = kStgOff + 8 * kStgWarpBytes;
   // kv_full[S], kv_empty[S], then per tile: q_full, q_empty, s_ready, p_ready,
-  // o_done, turn; then drain.
-  static constexpr int kNumBars = 2 * kStages + 6 * NQT + 1;
+  // o_done, turn; then drain; then per row quarter of each tile the two
+  // exchange barriers of a split row (x_up: part 1 -> part 0, x_down: back).
+  static constexpr int kNumBars = 2 * kStages + 6 * NQT + 1 + 2 * 4 * NQT;
   static constexpr int kCtlOff = kBarOff + kNumBars * 8;
-  static constexpr int kSmemBytes = kCtlOff + 64 + 1024;  // + runtime 1024-byte alignment
+  // Row-statistics exchange between the two threads of a row (SPLIT = 2):
+  // one float per query row of each tile.
+  static constexpr int kXOff = kCtlOff + 64;
+  static constexpr int kSmemBytes = kXOff + NQT * BM * 4 + 1024;  // + runtime 1024-byte alignment
   static constexpr uint32_t kOCol = 2 * BN;
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
@@ -251,17 +260,25 @@ __device__ __forceinline__ Item decode_item(int idx, const Params& p, int nkv_al
   return it;
 }
 
-// p = 2^(s * c - m) for one row of a score tile: writes P (rounded to T) to
-// tensor memory at tP, 32 columns at a time, and returns the fp32 sum of p.
-// POLY8 of every 8 columns use the polynomial exponential (only for tiles
-// without masked scores).
-template <typename T, int POLY8>
-__device__ __forceinline__ float exp_tile(const float (&s)[BN], float c, float m_use, uint32_t tP) {
+// Tensor-memory column (within S_t) of P for keys 16kk .. 16kk + 15.
+template <int SPLIT>
+__host__ __device__ constexpr uint32_t p_col(int kk) {
+  return SPLIT == 1 ? kPCol + kk * 8
+                    : static_cast<uint32_t>((kk / (BN / 16 / SPLIT)) * (BN / SPLIT) +
+                                            (kk % (BN / 16 / SPLIT)) * 8);
+}
+
+// p = 2^(s * c - m) for NC scores of one row: writes P (rounded to T) to
+// tensor memory at tP, 32 scores (16 columns) at a time, and returns the fp32
+// sum of p. POLY8 of every 8 columns use the polynomial exponential (only for
+// tiles without masked scores).
+template <typename T, int POLY8, int NC>
+__device__ __forceinline__ float exp_tile(const float (&s)[NC], float c, float m_use, uint32_t tP) {
   const uint64_t c2 = f2_make(c, c);
   const uint64_t nm2 = f2_make(-m_use, -m_use);
   uint64_t la = f2_make(0.f, 0.f), lb = la;
 #pragma unroll
-  for (int ch = 0; ch < BN / 32; ++ch) {
+  for (int ch = 0; ch < NC / 32; ++ch) {
     // 32 columns -> 16 packed words -> tensor memory, chunk by chunk so that
     // the registers of S are released as P is produced.
     uint32_t pk[16];
@@ -289,14 +306,18 @@ __device__ __forceinline__ float exp_tile(const float (&s)[BN], float c, float m
   return (a0 + a1) + (b0 + b1);
 }
 
-template <int D, typename T, bool CAUSAL, bool WINDOW, int POLY8, bool PINGPONG>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, typename T, bool CAUSAL, bool WINDOW, int POLY8, bool PINGPONG, int SPLIT = 1>
+__global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_o, const Params p) {
   using C = Cfg<D>;
   constexpr int S = C::kStages;
+  static_assert(SPLIT == 1 || (SPLIT == 2 && D == 128 && !PINGPONG), "row split");
+  constexpr int kMmaWarp = softmax_warps(SPLIT);
+  constexpr int kTmaWarp = kMmaWarp + 1;
+  constexpr int NC = BN / SPLIT;  // scores per softmax thread and key tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -313,6 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_done = p_ready + NQT;
   uint64_t* turn = o_done + NQT;
   uint64_t* drain = turn + NQT;
+  uint64_t* x_up = drain + 1;        // [NQT * 4]
+  uint64_t* x_down = x_up + 4 * NQT;  // [NQT * 4]
   CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem + C::kCtlOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kCtlOff + 32);
 
@@ -331,11 +354,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_full[t], 1);
       mbar_init(&q_empty[t], 1);
       mbar_init(&s_ready[t], 1);
-      mbar_init(&p_ready[t], 4 * 32);
+      mbar_init(&p_ready[t], 4 * 32 * SPLIT);
       mbar_init(&o_done[t], 1);
-      mbar_init(&turn[t], 4 * 32);
+      mbar_init(&turn[t], 4 * 32 * SPLIT);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 4 * NQT; ++i) {
+      mbar_init(&x_up[i], 32);
+      mbar_init(&x_down[i], 32);
+    }
     ctl->abort = 0;
     ctl->wait_ns = p.wait_ns;
     fence_mbar_init();
@@ -445,16 +472,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++pw[t];
             tc_fence_after();
             const uint32_t vd = v_lo + (((Lv % S) * C::kTileBytes) >> 4);
-            const uint32_t tP = tmem + t * BN + kPCol;
+            const uint32_t tS = tmem + t * BN;
             const uint32_t tO = tmem + C::kOCol + t * D;
-            // 16 keys = 16 rows of 128 bytes (2048 bytes = 128 in the address field)
+            // P of keys 16kk..16kk+15: 8 columns. With SPLIT = 1 P fills columns
+            // [64, 128) of S_t; with SPLIT = 2 the two halves of the row sit at
+            // columns [0, 32) and [64, 96), each where its own thread read S.
+            // 16 keys = 16 rows of 128 bytes of V (2048 bytes = 128 in the address field)
             if (j - 1 == s0)
-              umma_ts_w<0>(tO, tP, desc_words(vd, d_hi), idesc_pv);
+              umma_ts_w<0>(tO, tS + p_col<SPLIT>(0), desc_words(vd, d_hi), idesc_pv);
             else
-              umma_ts_w<1>(tO, tP, desc_words(vd, d_hi), idesc_pv);
+              umma_ts_w<1>(tO, tS + p_col<SPLIT>(0), desc_words(vd, d_hi), idesc_pv);
 #pragma unroll
             for (int kk = 1; kk < BN / 16; ++kk)
-              umma_ts_w<1>(tO, tP + kk * 8, desc_words(vd + kk * 128, d_hi), idesc_pv);
+              umma_ts_w<1>(tO, tS + p_col<SPLIT>(kk), desc_words(vd + kk * 128, d_hi), idesc_pv);
             if (j - 1 == n - 1) umma_commit_w(&o_done[t]);
           }
           if (j >= s0 && j < n) {
@@ -507,13 +537,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     drain_bar(drain, 0, ctl, kSiteDrain);
   } else {
     // ------------------------------------------------------------ softmax
-    const int t = warp >> 2;
+    // Warp w: query tile t = w / (4 SPLIT); row quarter q4 = w % 4 (the
+    // tensor-memory lanes a warp may access); column part hw = (w / 4) % SPLIT,
+    // i.e. scores [hw NC, (hw + 1) NC) of each of its 32 rows.
+    const int t = warp / (4 * SPLIT);
+    const int hw = (warp >> 2) % SPLIT;
     const int q4 = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * BN;
-    const uint32_t tP = tS + kPCol;
+    const uint32_t tS = tmem + lane_off + t * BN + hw * NC;
+    const uint32_t tP = tmem + lane_off + t * BN + p_col<SPLIT>(hw * (NC / 16));
     const uint32_t tO = tmem + lane_off + C::kOCol + t * D;
-    uint8_t* stg = smem + C::kStgOff + warp * C::kStgWarpBytes;  // this warp's O staging
+    uint8_t* stg = smem + C::kStgOff + (t * 4 + q4) * C::kStgWarpBytes;  // O staging (hw 0)
+    // Split rows: part 1 passes its tile max (then, at the end of an item, its
+    // partial row sum) up through xrow; part 0 returns the row max.
+    float* xrow = reinterpret_cast<float*>(smem + C::kXOff) + t * BM + q4 * 32 + lane;
+    uint64_t* xu = &x_up[t * 4 + q4];
+    uint64_t* xd = &x_down[t * 4 + q4];
+    uint32_t xp = 0;  // exchange rounds completed
     const float sl2 = p.scale_log2;
     uint32_t sw = 0;  // s_ready phases consumed
     uint32_t od = 0;  // o_done phases consumed
@@ -529,53 +569,65 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rt = it.r0 + t * BM;
       const int row = rt + q4 * 32 + lane;
       float m = -INFINITY;  // running max of s * c (log2 units)
-      float l = 0.f;        // running sum of p
+      float l = 0.f;        // running sum of p (this thread's columns)
       for (int i = s0; i < n; ++i) {
         if (!(ok = warp_all(wait_bar(&s_ready[t], sw & 1, ctl, kSiteSReady)))) break;
         ++sw;
         tc_fence_after();
-        uint32_t ra[32], rb[32], rc[32], rd[32];
-        tmem_ld_x32(tS + 0, ra);
-        tmem_ld_x32(tS + 32, rb);
-        tmem_ld_x32(tS + 64, rc);
-        tmem_ld_x32(tS + 96, rd);
-        tmem_wait_ld_x32(ra);
-        tmem_wait_ld_x32(rb);
-        tmem_wait_ld_x32(rc);
-        tmem_wait_ld_x32(rd);
-        float s[BN];
+        float s[NC];
+        {
+          uint32_t rr[NC / 32][32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          s[k] = __uint_as_float(ra[k]);
-          s[32 + k] = __uint_as_float(rb[k]);
-          s[64 + k] = __uint_as_float(rc[k]);
-          s[96 + k] = __uint_as_float(rd[k]);
+          for (int h = 0; h < NC / 32; ++h) tmem_ld_x32(tS + h * 32, rr[h]);
+#pragma unroll
+          for (int h = 0; h < NC / 32; ++h) tmem_wait_ld_x32(rr[h]);
+#pragma unroll
+          for (int h = 0; h < NC / 32; ++h)
+#pragma unroll
+            for (int k = 0; k < 32; ++k) s[h * 32 + k] = __uint_as_float(rr[h][k]);
         }
-        const int kv0 = (it.jb + i) * BN;
-        const bool edge = (CAUSAL && kv0 + BN - 1 > rt + p.off) || (kv0 + BN > p.Nk);
+        const int kv0 = (it.jb + i) * BN + hw * NC;  // key of s[0]
+        const bool edge = (CAUSAL && kv0 + NC - 1 > rt + p.off) || (kv0 + NC > p.Nk);
         if (edge) {
           const int last = (CAUSAL ? min(row + p.off, p.Nk - 1) : p.Nk - 1) - kv0;
 #pragma unroll
-          for (int k = 0; k < BN; ++k) s[k] = (k > last) ? -INFINITY : s[k];
+          for (int k = 0; k < NC; ++k) s[k] = (k > last) ? -INFINITY : s[k];
         }
         // Sliding window: keys before row + off - window + 1 are out of reach.
         const bool wedge = CAUSAL && WINDOW && kv0 < rt + BM + p.off - p.window;
         if (wedge) {
           const int first = row + p.off - p.window + 1 - kv0;
 #pragma unroll
-          for (int k = 0; k < BN; ++k) s[k] = (k < first) ? -INFINITY : s[k];
+          for (int k = 0; k < NC; ++k) s[k] = (k < first) ? -INFINITY : s[k];
         }
-        // four independent chains of 3-input max, 32 columns each
-        float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[32], s[33]);
-        float mx2 = fmaxf(s[64], s[65]), mx3 = fmaxf(s[96], s[97]);
+        // four independent chains of 3-input max, NC / 4 columns each
+        constexpr int Q = NC / 4;
+        float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[Q], s[Q + 1]);
+        float mx2 = fmaxf(s[2 * Q], s[2 * Q + 1]), mx3 = fmaxf(s[3 * Q], s[3 * Q + 1]);
 #pragma unroll
-        for (int k = 2; k < 32; k += 2) {
+        for (int k = 2; k < Q; k += 2) {
           mx0 = fmax3(mx0, s[k], s[k + 1]);
-          mx1 = fmax3(mx1, s[32 + k], s[33 + k]);
-          mx2 = fmax3(mx2, s[64 + k], s[65 + k]);
-          mx3 = fmax3(mx3, s[96 + k], s[97 + k]);
+          mx1 = fmax3(mx1, s[Q + k], s[Q + k + 1]);
+          mx2 = fmax3(mx2, s[2 * Q + k], s[2 * Q + k + 1]);
+          mx3 = fmax3(mx3, s[3 * Q + k], s[3 * Q + k + 1]);
         }
-        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        if (SPLIT == 2) {
+          // Both parts must scale the row by the same maximum.
+          if (hw == 1) {
+            *xrow = m_tile;
+            mbar_arrive(xu);
+            if (!(ok = warp_all(wait_bar(xd, xp & 1, ctl, kSiteXDown)))) break;
+            m_tile = *xrow;
+          } else {
+            if (!(ok = warp_all(wait_bar(xu, xp & 1, ctl, kSiteXUp)))) break;
+            m_tile = fmaxf(m_tile, *xrow);
+            *xrow = m_tile;
+            mbar_arrive(xd);
+          }
+          ++xp;
+        }
+        m_tile *= sl2;
         float alpha = 1.f;
         const bool need = m_tile > m + kRescaleThreshold;
         if (need) {
@@ -590,15 +642,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float lsum;
         if (POLY8 > 0 && !edge && !wedge)
-          lsum = exp_tile<T, POLY8>(s, sl2, m_use, tP);
+          lsum = exp_tile<T, POLY8, NC>(s, sl2, m_use, tP);
         else
-          lsum = exp_tile<T, 0>(s, sl2, m_use, tP);
+          lsum = exp_tile<T, 0, NC>(s, sl2, m_use, tP);
         l += lsum;
         if (PINGPONG) mbar_arrive(&turn[t ^ 1]);
         if (i > s0 && __any_sync(0xffffffffu, need)) {
-          // O_t was last written by PV_t(i-1), complete before S_t(i) was signalled.
+          // O_t was last written by PV_t(i-1), complete before S_t(i) was
+          // signalled. Each part of a split row rescales its share of the columns.
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = hw * (D / 32 / SPLIT); c < (hw + 1) * (D / 32 / SPLIT); ++c) {
             uint32_t o[32];
             tmem_ld_x32(tO + c * 32, o);
             tmem_wait_ld_x32(o);
@@ -631,6 +684,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       if (rt >= p.Nq) continue;  // no rows in this tile
+      if (SPLIT == 2) {
+        // Part 1 hands its partial row sum to part 0, which writes the row.
+        if (hw == 1) {
+          *xrow = l;
+          mbar_arrive(xu);
+          ok = warp_all(wait_bar(xd, xp & 1, ctl, kSiteXDown));
+          ++xp;
+          if (!ok) break;
+          continue;
+        }
+        if (!(ok = warp_all(wait_bar(xu, xp & 1, ctl, kSiteXUp)))) break;
+        l += *xrow;
+        mbar_arrive(xd);
+        ++xp;
+      }
       if (n > s0) {
         if (!(ok = warp_all(wait_bar(&o_done[t], od & 1, ctl, kSiteODone)))) break;
         ++od;
@@ -688,7 +756,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  if (warp < 8 && lane == 0) bulk_wait_group0();  // stores of O done before the CTA exits
+  // Stores of O done before the CTA exits (only part 0 of a row stores).
+  if (warp < kMmaWarp && ((warp >> 2) % SPLIT) == 0 && lane == 0) bulk_wait_group0();
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

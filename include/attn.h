@@ -207,6 +207,10 @@ int attn_merge_f16(float* o_acc, float* lse_acc, const void* o_part, const float
    (>= 1; always 1 for d other than 64 and 128), or a negative error code. */
 int attn_decode_num_splits(int B, int Hq, int Hkv, int d);
 
+/* The cudaError_t value (as an int) behind the calling thread's most recent
+   ATTN_ERR_CUDA from this library, or 0 if there was none. */
+int attn_last_cuda_error(void);
+
 /* Human-readable text for a return code. Never NULL. */
 const char* attn_strerror(int code);
 
