@@ -80,6 +80,8 @@ struct DParams {
   const int* seqlens;
   float* part_o;    // [nsplit][B][Hq][D]
   float* part_lse;  // [nsplit][B][Hq], log2 units
+  void* o;          // tensor-core split pass with nsplit == 1: the output itself, else NULL
+  float* lse;       //   and its LSE (natural log, may be NULL)
   int B;
   int Hq;
   int Hkv;

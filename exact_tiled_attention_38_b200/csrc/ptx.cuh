@@ -237,6 +237,32 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// ---------------------------------------------------------------- cp.async (16 bytes)
+// Copy 16 bytes global -> shared, of which the first src_bytes (0 or 16) are
+// read and the rest zero-filled: src_bytes = 0 reads nothing from global memory.
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the arrival is not counted in advance: the barrier's count includes it).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Order this thread's (generic-proxy) shared-memory accesses before later
+// async-proxy accesses (tcgen05.mma operand reads, bulk copies).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand.
 //   lbo / sbo: leading / stride byte offsets (multiples of 16).
 // For a K-major tile (rows of 128 bytes, 8-row swizzle atoms of 1024 bytes)

@@ -4,7 +4,9 @@ Covers the ragged GQA workload at full size (64 sequences, lengths uniform in
 [1024, 8192]) and small cases: length 1, empty sequences, lengths that are not
 multiples of the 32-key stage, MQA (one KV head for 32 query heads), MHA, a
 group of 3 (padded to 4), group 8, d = 64 and fp16, a single long sequence
-spread over many splits.
+spread over many splits; and, for the tensor-core split pass (groups of 8 to
+32 with d = 128), tile tails, padded groups, MQA, the workload's scale with
+groups of 8, and keys that move the running maximum at every tile.
 """
 import numpy as np
 import pytest
@@ -98,3 +100,67 @@ def test_decode_rejects_bad_arguments(lib):
     with pytest.raises(lib.AttnError) as e:
         lib.attn_decode(q, kc, kc, sl, Hkv=2, scale=float("nan"))
     assert e.value.code == lib.ATTN_ERR_INVALID
+
+
+# Groups of 8 to 32 query heads per KV head with d = 128 take the tensor-core
+# split pass (scores and P V as tcgen05 products, keys on tensor-memory lanes).
+TC_CASES = [
+    # B, Hq, Hkv, d, lengths, dtype
+    (4, 16, 2, 128, [1, 127, 128, 129], BF16),         # tile tails around 128 keys
+    (3, 32, 4, 128, [5000, 0, 260], F16),              # group 8, long + empty
+    (2, 32, 2, 128, [2049, 777], BF16),                # group 16 (no padding)
+    (2, 48, 2, 128, [1500, 300], BF16),                # group 24 (padded to 32)
+    (2, 32, 1, 128, [4100, 64], F16),                  # MQA, group 32
+    (64, 64, 8, 128, "ragged", BF16),                  # group 8 at the workload's scale
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: f"B{c[0]}h{c[1]}kv{c[2]}")
+def test_decode_tensor_core_groups(lib, case):
+    B, Hq, Hkv, d, lens, dt = case
+    if lens == "ragged":
+        sl = workloads.decode_seqlens(B, 1024, 8192, 2300)
+    else:
+        sl = torch.tensor(lens, dtype=torch.int32)
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, d, sl, dt,
+                                            seed=2100 + TC_CASES.index(case))
+    scale = d ** -0.5
+    o, lse = run(lib, q.to(DEV), kc.to(DEV), vc.to(DEV), sl.to(DEV), Hkv, scale)
+    o_ref, lse_ref = oracle.decode_ref(q, kc, vc, sl, scale, Hkv)
+    compare(o, lse, o_ref, lse_ref, dt, str(case[:4]))
+
+
+def test_decode_tensor_core_running_max_moves(lib):
+    # Keys grow along each sequence, so every 128-key tile raises the heads'
+    # maxima by far more than the lazy-rescale threshold (8 in log2 units) and
+    # the accumulated O^T is rescaled in tensor memory tile after tile.
+    B, Hq, Hkv, d = 2, 16, 2, 128
+    sl = torch.tensor([1300, 700], dtype=torch.int32)
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, d, sl, BF16, seed=2200)
+    rows = []
+    for b in range(B):
+        L = int(sl[b])
+        ramp = 1.0 + torch.arange(L, dtype=torch.float32) / 40.0
+        rows.append(ramp.repeat(Hkv))
+    kc = (kc.float().view(-1, d) * torch.cat(rows)[:, None]).to(BF16).view(kc.shape)
+    o, lse = run(lib, q.to(DEV), kc.to(DEV), vc.to(DEV), sl.to(DEV), Hkv, d ** -0.5)
+    o_ref, lse_ref = oracle.decode_ref(q, kc, vc, sl, d ** -0.5, Hkv)
+    compare(o, lse, o_ref, lse_ref, BF16, "growing keys")
+
+
+def test_decode_tensor_core_single_split_writes_output(lib):
+    # B * Hkv >= 2 waves of CTAs: one split per sequence, so the tensor-core
+    # pass writes O and LSE itself (no workspace, no combine). Includes empty
+    # and very short sequences, fp16, and the call without LSE.
+    B, Hq, Hkv, d = 40, 64, 8, 128
+    sl = workloads.decode_seqlens(B, 0, 300, 2400)
+    sl[3] = 0
+    sl[7] = 1
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, d, sl, F16, seed=2401)
+    assert lib.attn_decode_num_splits(B, Hq, Hkv, d) == 1
+    args = (q.to(DEV), kc.to(DEV), vc.to(DEV), sl.to(DEV), Hkv, d ** -0.5)
+    o, lse = run(lib, *args)
+    o_ref, lse_ref = oracle.decode_ref(q, kc, vc, sl, d ** -0.5, Hkv)
+    compare(o, lse, o_ref, lse_ref, F16, "single split")
+    o2, none = run(lib, *args, want_lse=False)
+    assert none is None and torch.equal(o, o2)
