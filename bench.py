@@ -42,10 +42,15 @@ PREFILL = workloads.PREFILL_MHA_2K
 DECODE = workloads.DECODE_GQA_RAGGED
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = [
-    os.path.join(ROOT, "exact_tiled_attention_38_b200", "csrc", f)
-    for f in ("prefill_sm100.cuh", "decode_sm100.cuh", "common.cuh", "ptx.cuh")
-]
+# Sources each measured kernel is compiled from (its traffic figure is valid
+# only while they hash to the value recorded with it).
+KERNEL_SOURCES = {
+    k: [os.path.join(ROOT, "exact_tiled_attention_38_b200", "csrc", f) for f in files]
+    for k, files in {
+        "attn_prefill_kernel": ("prefill_sm100.cuh", "common.cuh", "ptx.cuh"),
+        "attn_decode_split_kernel": ("decode_sm100.cuh", "common.cuh", "ptx.cuh"),
+    }.items()
+}
 
 
 # ----------------------------------------------------------------------------- accounting
@@ -88,9 +93,9 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in KERNEL_SOURCES[kernel]:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -105,7 +110,7 @@ def profiled_traffic(kernel: str):
     except (OSError, ValueError):
         return None
     ent = d.get(kernel)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 
