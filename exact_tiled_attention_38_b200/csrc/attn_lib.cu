@@ -176,6 +176,15 @@ int launch_fill_empty(void* o, float* lse, long long rows, int D, cudaStream_t s
 #define ETA_PREFILL_POLY8 0
 #endif
 
+// Prefill kernel knob: L2 prefetch of the next item's query tiles, issued by
+// the producer at the start of each item. Measured slower on B200 (2K causal
+// MHA 0.0840 ms against 0.0819 ms without, twice on one box; 32K causal GQA
+// unchanged): the producer decodes the next item and issues the prefetches
+// before the current item's own loads, which delays them.
+#ifndef ETA_PREFILL_PREFETCH_Q
+#define ETA_PREFILL_PREFETCH_Q 0
+#endif
+
 // Prefill kernel knob: softmax threads per query row for d = 128 (1 or 2).
 // Two threads per row (576-thread CTAs, 96 registers: five warps share an SM
 // sub-partition's register file) pass the same parity tests but measured about
@@ -191,7 +200,8 @@ template <int D, typename T, bool CAUSAL, bool WINDOW = false>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& to, const prefill::Params& p, int grid, cudaStream_t st) {
   constexpr int SPLIT = D == 128 ? ETA_PREFILL_SPLIT : 1;
-  auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, WINDOW, ETA_PREFILL_POLY8, false, SPLIT>;
+  auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, WINDOW, ETA_PREFILL_POLY8, false, SPLIT,
+                                           ETA_PREFILL_PREFETCH_Q != 0>;
   constexpr int smem = prefill::Cfg<D>::kSmemBytes;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
