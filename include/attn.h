@@ -111,7 +111,10 @@ int attn_fwd_f16(const void* q, const void* k, const void* v, void* o, float* ls
  * 256 MiB of freed blocks cached, so callers that synchronise between calls do
  * not pay for re-mapping device memory each time. The caller's pools are not
  * touched. Other d use one block per (sequence, query head), no split and no
- * scratch.
+ * scratch. With d = 128 and 8 to 32 query heads per KV head the split pass runs
+ * on the tensor cores; when it uses one split per sequence
+ * (attn_decode_num_splits returns 1) it writes o and lse itself and nothing is
+ * allocated.
  */
 int attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
                 void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
