@@ -177,10 +177,10 @@ int launch_fill_empty(void* o, float* lse, long long rows, int D, cudaStream_t s
 #endif
 
 // Prefill kernel knob: L2 prefetch of the next item's query tiles, issued by
-// the producer at the start of each item. Measured slower on B200 (2K causal
-// MHA 0.0840 ms against 0.0819 ms without, twice on one box; 32K causal GQA
-// unchanged): the producer decodes the next item and issues the prefetches
-// before the current item's own loads, which delays them.
+// the producer right after the current item's own query loads. Measured
+// slower on B200 on the 2K causal MHA workload, whether issued before or after
+// those loads (0.0840 ms against 0.0819 ms without, in interleaved runs on one
+// box; 32K causal GQA within noise), so it is off.
 #ifndef ETA_PREFILL_PREFETCH_Q
 #define ETA_PREFILL_PREFETCH_Q 0
 #endif

@@ -393,21 +393,6 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
         const int idx = item_index(r, cta, G);
         if (idx >= p.total) break;
         const Item it = decode_item<CAUSAL, WINDOW>(idx, p, nkv_all);
-        if (PREFETCH_Q) {
-          // The next item's Q tiles are read once, from HBM: start them into
-          // L2 now, so that their loads (issued only when this item's last
-          // score products have read the current tiles) hit L2.
-          const int nidx = item_index(r + 1, cta, G);
-          if (nidx < p.total) {
-            const Item nx = decode_item<CAUSAL, WINDOW>(nidx, p, nkv_all);
-#pragma unroll
-            for (int t = 0; t < NQT; ++t) {
-              if ((t ? nx.n1 - nx.s1 : nx.n0 - nx.s0) <= 0) continue;
-              for (int bx = 0; bx < C::kBoxes; ++bx)
-                tma_prefetch_l2_3d(&tm_q, bx * 64, nx.r0 + t * BM, nx.bh);
-            }
-          }
-        }
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
           if ((t ? it.n1 - it.s1 : it.n0 - it.s0) <= 0) continue;
@@ -418,6 +403,22 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
             tma_load_3d(sQ + t * C::kTileBytes + bx * C::kBoxBytes, &tm_q, &q_full[t], bx * 64,
                         it.r0 + t * BM, it.bh);
           ++qn[t];
+        }
+        if (PREFETCH_Q) {
+          // The next item's Q tiles are read once, from HBM: start them into
+          // L2 now (after this item's own Q loads), so that their loads,
+          // issued only when this item's last score products have read the
+          // current tiles, hit L2.
+          const int nidx = item_index(r + 1, cta, G);
+          if (nidx < p.total) {
+            const Item nx = decode_item<CAUSAL, WINDOW>(nidx, p, nkv_all);
+#pragma unroll
+            for (int t = 0; t < NQT; ++t) {
+              if ((t ? nx.n1 - nx.s1 : nx.n0 - nx.s0) <= 0) continue;
+              for (int bx = 0; bx < C::kBoxes; ++bx)
+                tma_prefetch_l2_3d(&tm_q, bx * 64, nx.r0 + t * BM, nx.bh);
+            }
+          }
         }
         const int nmax = max(it.n0, it.n1);
         const int zkv = it.b * p.Hkv + it.kvh;
