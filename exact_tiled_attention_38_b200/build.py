@@ -13,10 +13,12 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG_DIR)
 SRC = os.path.join(PKG_DIR, "csrc", "attn_lib.cu")
 OUT = os.path.join(PKG_DIR, "libattn.so")
-DEPS = [
+# Every source the library is compiled from: all of csrc/ and the header.
+DEPS = sorted(
     os.path.join(PKG_DIR, "csrc", f)
-    for f in ("attn_lib.cu", "common.cuh", "ptx.cuh", "prefill_sm100.cuh", "decode_sm100.cuh")
-] + [os.path.join(ROOT, "include", "attn.h")]
+    for f in os.listdir(os.path.join(PKG_DIR, "csrc"))
+    if f.endswith((".cu", ".cuh", ".h"))
+) + [os.path.join(ROOT, "include", "attn.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -161,3 +161,11 @@ def test_merge_host_validation(clib):
     assert merge(la=ctypes.c_void_p(0x10002)) == eta.ATTN_ERR_INVALID
     assert merge(out=ctypes.c_void_p(0x10004)) == eta.ATTN_ERR_INVALID
     assert clib.attn_merge_f16(FAKE, FAKE, FAKE, FAKE, None, 0, 64, None) == eta.ATTN_OK
+
+
+def test_build_tracks_every_source():
+    # A change to any kernel source must trigger a rebuild of the library.
+    csrc = os.path.join(ROOT, "exact_tiled_attention_38_b200", "csrc")
+    srcs = {os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh"))}
+    assert srcs <= set(eta_build.DEPS)
+    assert HEADER in eta_build.DEPS
