@@ -67,3 +67,14 @@ def test_noalloc_refuses_sizes_beyond_its_scratch(lib):
     with pytest.raises(lib.AttnError) as e:
         lib.attn_decode_noalloc(q, kc, kc, sl, Hkv=Hkv)
     assert e.value.code == lib.ATTN_ERR_SCRATCH
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,lens", [
+    (3, 32, 4, [2000, 10, 700]),   # tensor-core split pass, several splits in the scratch
+    (40, 64, 8, None),             # tensor-core pass, one split: writes o and lse itself
+])
+def test_noalloc_tensor_core_groups(lib, B, Hq, Hkv, lens):
+    sl = torch.tensor(lens, dtype=torch.int32) if lens else workloads.decode_seqlens(B, 0, 400, 41)
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, 128, sl, torch.bfloat16, seed=43,
+                                            device=DEV)
+    _call_pair(lib, q, kc, vc, sl, Hkv)
