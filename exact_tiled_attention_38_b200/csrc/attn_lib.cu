@@ -1,6 +1,12 @@
 // C-ABI boundary of the attention library: argument checks, TMA descriptor
-// encoding, launch configuration and error codes. Every step of the
-// computation runs in the kernels of prefill_sm100.cuh and decode_sm100.cuh.
+// encoding, kernel selection, launch configuration and error codes. Every
+// step of the computation runs in the kernels:
+//   prefill_sm100.cuh    prefill, d = 64 / 128 (tcgen05, TMA)
+//   decode_sm100.cuh     decode split pass on CUDA cores (d = 64, groups <= 4)
+//                        and the LSE combine
+//   decode_tc_sm100.cuh  decode split pass on tcgen05 (d = 128, groups 8..32)
+//   generic_fwd.cuh      prefill and decode for the other head sizes
+//   merge.cuh            LSE merge of partial results (context parallelism)
 #include <cuda.h>
 #include <cuda_runtime.h>
 
