@@ -191,12 +191,6 @@ int launch_fill_empty(void* o, float* lse, long long rows, int D, cudaStream_t s
 #define ETA_PREFILL_PREFETCH_Q 0
 #endif
 
-// Prefill kernel knob: issue the next item's first score product for query
-// tile 0 during the current item's last iteration (causal, no window).
-#ifndef ETA_PREFILL_EARLY_S0
-#define ETA_PREFILL_EARLY_S0 0
-#endif
-
 // Prefill kernel knob: softmax threads per query row for d = 128 (1 or 2).
 // Two threads per row (576-thread CTAs, 96 registers: five warps share an SM
 // sub-partition's register file) pass the same parity tests but measured about
@@ -213,7 +207,7 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
                    const CUtensorMap& to, const prefill::Params& p, int grid, cudaStream_t st) {
   constexpr int SPLIT = D == 128 ? ETA_PREFILL_SPLIT : 1;
   auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, WINDOW, ETA_PREFILL_POLY8, false, SPLIT,
-                                           ETA_PREFILL_PREFETCH_Q != 0, ETA_PREFILL_EARLY_S0 != 0>;
+                                           ETA_PREFILL_PREFETCH_Q != 0>;
   constexpr int smem = prefill::Cfg<D>::kSmemBytes;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;

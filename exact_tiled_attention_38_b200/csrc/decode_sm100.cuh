@@ -20,11 +20,6 @@
 //   combine      one warp per (b, query head): merges the partials by their
 //                log-sum-exp and writes O (input dtype) and LSE (natural log).
 //
-// This CUDA-core split pass serves d = 64 and groups of up to 4 query heads per
-// KV head (larger groups are split into chunks of 4); for d = 128 and groups of
-// 8 to 32 the tensor-core split pass of decode_tc_sm100.cuh takes its place and
-// feeds the same combine.
-//
 // Packed cache layout: sequence b starts at token offset sum_{j<b} L_j and is
 // stored [Hkv][L_b][d], so one (sequence, KV head) is one contiguous run. The
 // offsets are recomputed on the device from `seqlens`; negative lengths count
@@ -54,8 +49,7 @@ enum : unsigned { kSiteStage = 0x21, kSiteDrain = 0x22 };
 #define ETA_DECODE_STAGES 3
 #endif
 
-// GP: query heads per CTA (the group, padded up to 4; 8 only with the
-// ETA_DECODE_MAX_GP=8 build knob).
+// GP: query heads per CTA (the group, padded up to 4 or 8).
 template <int D, int GP>
 struct DCfg {
   static_assert(D == 64 || D == 128, "head dim");

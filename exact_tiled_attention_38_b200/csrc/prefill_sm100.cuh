@@ -307,7 +307,7 @@ __device__ __forceinline__ float exp_tile(const float (&s)[NC], float c, float m
 }
 
 template <int D, typename T, bool CAUSAL, bool WINDOW, int POLY8, bool PINGPONG, int SPLIT = 1,
-          bool PREFETCH_Q = false, bool EARLY_S0 = false>
+          bool PREFETCH_Q = false>
 __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -462,56 +462,15 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
     int qi[NQT] = {0, 0};
     uint32_t pw[NQT] = {0, 0};
     bool ok = true;
-    // Causal items pair query tiles with n and n + 1 key tiles, so tile 0 has
-    // no product in an item's last iteration. With EARLY_S0 the next item's
-    // first score product for tile 0 is issued there, before the wait for tile
-    // 1's last probabilities: tile 0's softmax group starts the next item
-    // while tile 1 finishes this one, instead of both restarting together.
-    // Its Q tile was loaded after tile 0's last product of this item, its K
-    // tile follows this item's last V tile in the ring (that stage was freed
-    // two iterations earlier), and P_0 of this item was consumed by a P V
-    // product issued before it.
-    constexpr bool kEarly = EARLY_S0 && CAUSAL && !WINDOW;
-    bool s0_issued = false;  // this item's S_0(0) was issued during the previous item
     for (int r = 0; ok; ++r) {
       const int idx = item_index(r, cta, G);
       if (idx >= p.total) break;
       const Item it = decode_item<CAUSAL, WINDOW>(idx, p, nkv_all);
       const int nmax = max(it.n0, it.n1);
-      bool s0_next = false;
       for (int j = 0; ok && j <= nmax; ++j) {
         const uint32_t Lk = L + 2 * j;
         const uint32_t Lv = L + 2 * j - 1;
-        bool have_k = kEarly && j == 0 && s0_issued;  // K_0 was waited for then
-        if (kEarly && j == nmax && it.n0 < nmax) {
-          const int nidx = item_index(r + 1, cta, G);
-          if (nidx < p.total) {
-            const Item nx = decode_item<CAUSAL, WINDOW>(nidx, p, nkv_all);
-            if (nx.n0 > 0) {
-              const uint32_t Ln = L + 2 * nmax;  // the next item's K_0
-              const int qph = qi[0] + (it.n0 > it.s0 ? 1 : 0);
-              if (!(ok = warp_all(wait_bar(&kv_full[Ln % S], (Ln / S) & 1, ctl, kSiteKvFull))))
-                break;
-              if (!(ok = warp_all(wait_bar(&q_full[0], qph & 1, ctl, kSiteQFull)))) break;
-              tc_fence_after();
-              const uint32_t kd = k_lo + (((Ln % S) * C::kTileBytes) >> 4);
-#pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
-                if (kk == 0)
-                  umma_ss_w<0>(tmem, desc_words(q_lo + koff, d_hi), desc_words(kd + koff, d_hi),
-                               idesc_s);
-                else
-                  umma_ss_w<1>(tmem, desc_words(q_lo + koff, d_hi), desc_words(kd + koff, d_hi),
-                               idesc_s);
-              }
-              umma_commit_w(&s_ready[0]);
-              if (nx.n0 == 1) umma_commit_w(&q_empty[0]);
-              s0_next = true;
-            }
-          }
-        }
-        bool have_v = false;
+        bool have_k = false, have_v = false;
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
           if (!ok) break;
@@ -545,9 +504,7 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
               umma_ts_w<1>(tO, tS + p_col<SPLIT>(kk), desc_words(vd + kk * 128, d_hi), idesc_pv);
             if (j - 1 == n - 1) umma_commit_w(&o_done[t]);
           }
-          if (kEarly && t == 0 && j == 0 && s0_issued) {
-            // S_0(0) already issued (and q_empty committed if it was the last)
-          } else if (j >= s0 && j < n) {
+          if (j >= s0 && j < n) {
             // S_t = Q_t K_j^T
             if (!have_k) {
               if (!(ok = warp_all(wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull))))
@@ -591,7 +548,6 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
       L += 2 * nmax;
       qi[0] += it.n0 > it.s0;
       qi[1] += it.n1 > it.s1;
-      s0_issued = s0_next;
     }
     // Every MMA must be complete before tensor memory is released.
     umma_commit_w(drain);
