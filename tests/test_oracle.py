@@ -531,3 +531,47 @@ def test_window_pins_catch_an_off_by_one(monkeypatch):
         test_window_matches_brute_force(7, 7, 3)
     with pytest.raises(AssertionError):
         test_window_one_key_returns_that_value()
+
+
+# Property sweep: random shapes, groupings, lengths and scales against the
+# library routine (fp64 torch SDPA with a bottom-right causal mask).
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None)
+@given(B=st.integers(1, 2), Hkv=st.integers(1, 3), group=st.integers(1, 4),
+       Nq=st.integers(1, 17), Nk=st.integers(1, 17), d=st.sampled_from([4, 8, 16]),
+       causal=st.booleans(), scale=st.floats(0.05, 2.0), seed=st.integers(0, 10_000))
+def test_property_sweep_matches_torch_sdpa(B, Hkv, group, Nq, Nk, d, causal, scale, seed):
+    if causal and Nq > Nk:
+        Nq, Nk = Nk, Nq  # every causal row keeps at least its diagonal key
+    Hq = Hkv * group
+    q = _rand((B, Hq, Nq, d), seed)
+    k = _rand((B, Hkv, Nk, d), seed + 1)
+    v = _rand((B, Hkv, Nk, d), seed + 2)
+    o, lse = oracle.attention_ref(q, k, v, scale, causal)
+    assert np.abs(o - _sdpa(q, k, v, scale, causal).numpy()).max() < TOL
+    assert np.abs(lse - _lse_lib(q, k, scale, causal).numpy()).max() < TOL
+
+
+@settings(max_examples=40, deadline=None)
+@given(Hkv=st.integers(1, 2), group=st.integers(1, 3), Nq=st.integers(1, 15),
+       extra=st.integers(0, 10), W=st.integers(1, 20), seed=st.integers(0, 10_000))
+def test_property_sweep_window_matches_banded_sdpa(Hkv, group, Nq, extra, W, seed):
+    # The window as an explicit band of the score matrix handed to SDPA:
+    # row i keeps keys j with i + off - W < j <= i + off, off = Nk - Nq >= 0.
+    Nk = Nq + extra
+    Hq, d, scale = Hkv * group, 8, 0.4
+    q = _rand((1, Hq, Nq, d), seed)
+    k = _rand((1, Hkv, Nk, d), seed + 1)
+    v = _rand((1, Hkv, Nk, d), seed + 2)
+    i = torch.arange(Nq)[:, None] + extra
+    j = torch.arange(Nk)[None, :]
+    band = (j <= i) & (j > i - W)
+    ref = F.scaled_dot_product_attention(q, k, v, attn_mask=band, scale=scale,
+                                         enable_gqa=group > 1)
+    kr = k.repeat_interleave(group, dim=1)
+    s = (scale * (q @ kr.transpose(-1, -2))).masked_fill(~band, float("-inf"))
+    o, lse = oracle.attention_ref(q, k, v, scale, True, window=W)
+    assert np.abs(o - ref.numpy()).max() < TOL
+    assert np.abs(lse - torch.logsumexp(s, dim=-1).numpy()).max() < TOL
