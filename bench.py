@@ -41,6 +41,9 @@ METRIC = "prefill attn TFLOP/s & decode KV-cache GB/s, as % of B200 roofline"
 PREFILL = workloads.PREFILL_MHA_2K
 DECODE = workloads.DECODE_GQA_RAGGED
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Spec-sheet figures for one B200, for context beside the measured peaks: dense
+# bf16 tensor throughput (without 2:4 sparsity) and HGX HBM3e bandwidth.
+NOMINAL_PEAKS = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 # Sources each measured kernel is compiled from (its traffic figure is valid
 # only while they hash to the value recorded with it).
@@ -294,6 +297,51 @@ def cpu_baseline(budget_s: float = 12.0):
     }
 
 
+def run_oracle_timing(budget_s: float = 10.0) -> int:
+    """CPU only: the fp64 oracle, as it stands, on the small fp16 workload (whole)
+    and on the 32K and 128K causal GQA workloads (a bounded set of query rows of
+    one head, with the time for every row of every head extrapolated from the
+    oracle's own cost per row, which is proportional to Nk: it scores a row
+    against every key and then masks). Inputs have the workloads' shapes; the
+    timing does not depend on their values. One JSON line per workload."""
+    import torch
+
+    import oracle
+
+    cores = blas_threads()
+    w0 = workloads.PREFILL_SMALL
+    q, k, v = workloads.prefill_inputs(w0, device="cpu")
+    t0 = time.perf_counter()
+    oracle.attention_ref(q, k, v, w0.scale, w0.causal)
+    sec = time.perf_counter() - t0
+    print(json.dumps({"variant": f"oracle_cpu_{w0.name}", "kind": "oracle", "cores": cores,
+                      "sample": "whole workload", "seconds": round(sec, 4),
+                      "value": round(prefill_flops(w0) / sec / 1e9, 3), "unit": "GFLOP/s"}),
+          flush=True)
+    for w in (workloads.PREFILL_GQA_32K, workloads.PREFILL_GQA_128K):
+        gen = torch.Generator().manual_seed(w.seed)
+        kh = torch.randn(1, 1, w.Nk, w.d, generator=gen).to(torch.bfloat16)
+        vh = torch.randn(1, 1, w.Nk, w.d, generator=gen).to(torch.bfloat16)
+        rows, spent = [], 0.0
+        rng = np.random.default_rng(w.seed + 100)
+        while spent < budget_s / 2 and len(rows) < w.Nq:
+            r = int(rng.integers(0, w.Nq))
+            qh = torch.randn(1, 1, 1, w.d, generator=gen).to(torch.bfloat16)
+            t0 = time.perf_counter()
+            oracle.attention_ref(qh, kh, vh, w.scale, w.causal, rows=[r], nq=w.Nq)
+            spent += time.perf_counter() - t0
+            rows.append(r)
+        full_rows = w.B * w.Hq * w.Nq
+        print(json.dumps({
+            "variant": f"oracle_cpu_{w.name}", "kind": "oracle", "cores": cores,
+            "sample": f"{len(rows)} query rows of one head against all {w.Nk} keys",
+            "seconds": round(spent, 3),
+            "extrapolated_full_seconds": round(spent / len(rows) * full_rows, 1),
+            "extrapolation": "per-row time x every row of every head (cost per row ~ Nk)"}),
+            flush=True)
+    return 0
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -506,13 +554,17 @@ def run_ours(args, world, rank, local):
                      "kernel": "attn_decode_split_kernel<128,4,bf16> + attn_decode_combine_kernel"
                                " (one attn_decode call, timed together)",
                      "algorithmic_bytes": dbytes, "ms_per_launch": dec_ms,
-                     "peak_source": f"{src} copy bandwidth (burst)"},
+                     "peak_source": f"{src} copy bandwidth (burst)",
+                     "nominal": {"peak": NOMINAL_PEAKS["hbm_gbs"],
+                                 "frac": dec_ach / NOMINAL_PEAKS["hbm_gbs"]}},
         "roofline_prefill": {"bound": "tensor", "achieved": pre_ach, "peak": peaks["bf16_tflops"],
                              "unit": "TFLOP/s", "frac": pre_ach / peaks["bf16_tflops"],
                              "traffic": profiled_traffic("attn_prefill_kernel"),
                              "kernel": "attn_prefill_kernel<128,bf16,causal>",
                              "algorithmic_flops": flops, "ms_per_launch": pre_ms,
-                             "peak_source": f"{src} bf16 dense matmul (burst)"},
+                             "peak_source": f"{src} bf16 dense matmul (burst)",
+                             "nominal": {"peak": NOMINAL_PEAKS["bf16_tflops"],
+                                         "frac": pre_ach / NOMINAL_PEAKS["bf16_tflops"]}},
         "decode": {"value": dec_gbs, "unit": "GB/s (KV cache read)", "ms_per_call": dec_ms},
         "e2e": {"value": aggregate_throughput(flops, world, e2e_pre) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -716,12 +768,17 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=("prefill", "prefill_32k", "decode"), default=None,
                     help="only launch this phase (an ncu target); prints nothing")
+    ap.add_argument("--oracle-timing", action="store_true",
+                    help="CPU only: time the fp64 oracle on the small, 32K and 128K workloads "
+                         "(sampled rows, extrapolated)")
     ap.add_argument("--variants", action="store_true",
                     help="measure the extra shapes (long context, head groupings, d, dtype), "
                          "one JSON line each, instead of the step")
     args = ap.parse_args(argv)
     if args.warmup < 3 and not args.profile:
         ap.error("--warmup must be >= 3")
+    if args.oracle_timing:
+        return run_oracle_timing()
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, world, rank)
