@@ -443,6 +443,7 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale) || window < 0)
     return ATTN_ERR_INVALID;
   if (!tensor_core_d(d) && !generic_d(d)) return ATTN_ERR_UNSUPPORTED;
+  if (tensor_core_d(d) && B > 65535) return ATTN_ERR_UNSUPPORTED;  // one grid z slice per sequence
   if (static_cast<long long>(B) * Hq > 0x7fffffffLL / 4) return ATTN_ERR_INVALID;
   if (B == 0) return ATTN_OK;
   if (q == nullptr || kc == nullptr || vc == nullptr || seqlens == nullptr || o == nullptr ||
@@ -709,6 +710,7 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
                        cudaStream_t st) {
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || !scale_ok(scale)) return ATTN_ERR_INVALID;
   if (!tensor_core_d(d) && !generic_d(d)) return ATTN_ERR_UNSUPPORTED;
+  if (tensor_core_d(d) && B > 65535) return ATTN_ERR_UNSUPPORTED;  // one grid z slice per sequence
   if (static_cast<long long>(B) * Hq > 0x7fffffffLL / 4) return ATTN_ERR_INVALID;
   if (B == 0) return ATTN_OK;
   if (q == nullptr || kc == nullptr || vc == nullptr || seqlens == nullptr || o == nullptr ||

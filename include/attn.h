@@ -77,7 +77,7 @@ enum attn_status {
  *                (equal to the usual lower-triangular mask when Nq == Nk).
  * Sizes: B >= 0, Nq >= 0, Nk >= 0 (B == 0 or Nq == 0: nothing to do;
  * Nk == 0: every row is empty), Hq >= 1, Hkv >= 1, Hq % Hkv == 0,
- * d a multiple of 8 in [8, 256], Nq <= 16,776,960 (generic d: B * Hq <= 65,535).
+ * d a multiple of 8 in [8, 256], Nq <= 16,776,960, B * Hq < 2^31.
  * Allocates no device memory.
  */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -103,7 +103,8 @@ int attn_fwd_f16(const void* q, const void* k, const void* v, void* o, float* ls
  *           values count as 0; 0 gives o = 0, lse = -inf).
  *   o       [B, Hq, d]  bf16       lse [B, Hq] float32 (or NULL)
  * Sizes: B >= 0 (0: nothing to do), Hq >= 1, Hkv >= 1, Hq % Hkv == 0,
- * d a multiple of 8 in [8, 256] (generic d: B * Hq <= 65,535).
+ * d a multiple of 8 in [8, 256], B * Hq < 2^29; for d = 64 and 128 also
+ * B <= 65,535 (larger B returns ATTN_ERR_UNSUPPORTED).
  * For d = 64 and 128, allocates a split-KV scratch of nsplit * B * Hq * (d + 1) * 4 bytes with
  * cudaMallocFromPoolAsync on `stream` and frees it with cudaFreeAsync on the
  * same stream (stream-ordered; no block outlives the call's work). The pool is

@@ -169,3 +169,10 @@ def test_build_tracks_every_source():
     srcs = {os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh"))}
     assert srcs <= set(eta_build.DEPS)
     assert HEADER in eta_build.DEPS
+
+
+def test_decode_batch_limit_of_the_split_passes(clib):
+    # d = 64 / 128 decode launches one grid z slice per sequence
+    assert dec(clib, B=65536, Hq=1, Hkv=1) == eta.ATTN_ERR_UNSUPPORTED
+    assert clib.attn_decode_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, None, 65536, 1, 1, 128, 0.1,
+                                    None) == eta.ATTN_ERR_UNSUPPORTED
