@@ -57,6 +57,26 @@ inline int launch_status() {
   return e == cudaSuccess ? ATTN_OK : cuda_fail(e);
 }
 
+// A setup step (a kernel attribute) done once per device and remembered: the
+// attribute applies to the current device only, so a process that drives
+// several GPUs needs it on each.
+struct PerDeviceOnce {
+  std::mutex mu;
+  bool done[64] = {};
+  cudaError_t err[64] = {};
+  template <typename F>
+  cudaError_t run(F&& step) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+      err[dev] = step();
+      done[dev] = true;
+    }
+    return err[dev];
+  }
+};
+
 struct DeviceInfo {
   int sm_count = 0;
   bool sm100 = false;
@@ -209,10 +229,9 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, WINDOW, ETA_PREFILL_POLY8, false, SPLIT,
                                            ETA_PREFILL_PREFETCH_Q != 0>;
   constexpr int smem = prefill::Cfg<D>::kSmemBytes;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&]() {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static PerDeviceOnce attr;
+  const cudaError_t attr_err = attr.run([&]() {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err);
   kern<<<grid, prefill::kernel_threads(SPLIT), smem, st>>>(tq, tk, tv, to, p);
@@ -356,10 +375,9 @@ template <int D, int GP, typename T>
 int launch_decode_split(const decode::DParams& p, cudaStream_t st) {
   auto kern = decode::attn_decode_split_kernel<D, GP, T>;
   constexpr int smem = decode::DCfg<D, GP>::kSmemBytes;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&]() {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static PerDeviceOnce attr;
+  const cudaError_t attr_err = attr.run([&]() {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err);
   const dim3 grid(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(p.Hkv * p.nchunk),
@@ -372,10 +390,9 @@ template <int NP, typename T>
 int launch_decode_tc(const decode::DParams& p, cudaStream_t st) {
   auto kern = decode_tc::attn_decode_tc_kernel<NP, T>;
   constexpr int smem = decode_tc::TCfg<NP>::kSmemBytes;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&]() {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static PerDeviceOnce attr;
+  const cudaError_t attr_err = attr.run([&]() {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err);
   const dim3 grid(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(p.Hkv),
