@@ -101,6 +101,18 @@ def _dev(t, name):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _on_device(*tensors):
+    """The library works on the current CUDA device: every tensor of a call must
+    live on one device, which is made current for the call (and whose current
+    stream is used when none is given)."""
+    import torch
+
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"all tensors of a call must be on one CUDA device, got {sorted(map(str, devs))}")
+    return torch.cuda.device(next(iter(devs)))
+
+
 def _fwd(fname, dtype, q, k, v, o, lse, scale, causal, stream, want_lse, window=None):
     import torch
 
@@ -126,10 +138,11 @@ def _fwd(fname, dtype, q, k, v, o, lse, scale, causal, stream, want_lse, window=
         if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Nq):
             raise ValueError("lse must be float32 [B, Hq, Nq]")
     fn = getattr(load_library(), fname)
-    code = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-              lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
-              float(scale), *((int(window),) if window is not None else (1 if causal else 0,)),
-              _stream_handle(stream))
+    with _on_device(q, k, v, o, lse):
+        code = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                  lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
+                  float(scale), *((int(window),) if window is not None else (1 if causal else 0,)),
+                  _stream_handle(stream))
     _check(code, fname)
     return o, lse
 
@@ -174,10 +187,11 @@ def _decode(fname, dtype, q, kcache, vcache, seqlens, Hkv, o, lse, scale, stream
     if lse is None and want_lse:
         lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
     fn = getattr(load_library(), fname)
-    code = fn(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
-              o.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, d,
-              float(scale), *((int(window),) if window is not None else ()),
-              _stream_handle(stream))
+    with _on_device(q, kcache, vcache, seqlens, o, lse):
+        code = fn(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
+                  o.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, d,
+                  float(scale), *((int(window),) if window is not None else ()),
+                  _stream_handle(stream))
     _check(code, fname)
     return o, lse
 
@@ -265,9 +279,10 @@ def attn_merge(o_acc, lse_acc, o_part, lse_part, o_out=None, stream=None) -> Non
             raise ValueError("o_out must match o_part")
     name = "attn_merge_f16" if o_part.dtype == torch.float16 else "attn_merge"
     rows = o_part.numel() // d if d else 0
-    code = getattr(load_library(), name)(
-        o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
-        o_out.data_ptr() if o_out is not None else None, rows, d, _stream_handle(stream))
+    with _on_device(o_acc, lse_acc, o_part, lse_part, o_out):
+        code = getattr(load_library(), name)(
+            o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+            o_out.data_ptr() if o_out is not None else None, rows, d, _stream_handle(stream))
     _check(code, name)
 
 

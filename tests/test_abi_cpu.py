@@ -176,3 +176,15 @@ def test_decode_batch_limit_of_the_split_passes(clib):
     assert dec(clib, B=65536, Hq=1, Hkv=1) == eta.ATTN_ERR_UNSUPPORTED
     assert clib.attn_decode_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, None, 65536, 1, 1, 128, 0.1,
                                     None) == eta.ATTN_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_tensors_on_different_devices():
+    import torch
+
+    class FakeDev:  # stands in for CUDA tensors on two devices (no GPU needed)
+        def __init__(self, dev):
+            self.device = torch.device(dev)
+
+    with pytest.raises(ValueError):
+        eta._on_device(FakeDev("cuda:0"), FakeDev("cuda:1"))
+    eta._on_device(FakeDev("cuda:1"), None, FakeDev("cuda:1"))  # one device: fine
