@@ -177,3 +177,28 @@ def test_ring_exchange_over_gloo(world, causal):
     assert sorted(r for r, _, _ in res) == list(range(world))
     for rank, err_o, err_l in res:
         assert err_o < 1e-6 and err_l < 1e-6, (rank, err_o, err_l)
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(world=st.integers(1, 4), c=st.integers(1, 5), Hkv=st.integers(1, 2),
+       group=st.integers(1, 3), causal=st.booleans(), seed=st.integers(0, 1000))
+def test_property_ring_matches_full_oracle(world, c, Hkv, group, causal, seed):
+    # Any world size and chunk length: every rank's output, put back in order,
+    # equals the oracle over the whole sequence.
+    N, d = 2 * world * c, 8
+    q, k, v = _inputs(1, Hkv * group, Hkv, N, d, seed=seed)
+    ks = [cp.shard_zigzag(k, r, world) for r in range(world)]
+    vs = [cp.shard_zigzag(v, r, world) for r in range(world)]
+    outs, lses = [], []
+    for r in range(world):
+        ex = cp.LocalRing(r, ks, vs) if world > 1 else None
+        o, lse = cp.ring_attention(cp.shard_zigzag(q, r, world), ks[r], vs[r], causal, 0.3,
+                                   exchange=ex, ops=OracleOps())
+        outs.append(o)
+        lses.append(lse)
+    o_ref, lse_ref = oracle.attention_ref(q, k, v, 0.3, causal)
+    np.testing.assert_allclose(cp.unshard_zigzag(outs).numpy(), o_ref, atol=1e-6, rtol=0)
+    np.testing.assert_allclose(cp.unshard_zigzag(lses).numpy(), lse_ref, atol=1e-6, rtol=0)
