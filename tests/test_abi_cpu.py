@@ -188,3 +188,28 @@ def test_binding_refuses_tensors_on_different_devices():
     with pytest.raises(ValueError):
         eta._on_device(FakeDev("cuda:0"), FakeDev("cuda:1"))
     eta._on_device(FakeDev("cuda:1"), None, FakeDev("cuda:1"))  # one device: fine
+
+
+def test_header_is_plain_c_and_links(tmp_path, clib):
+    # The boundary is a C ABI: the header compiles as C99 with warnings as
+    # errors, and a C program that takes the address of every entry point links
+    # against the library.
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    names = declared_functions()
+    src = tmp_path / "abi.c"
+    src.write_text('#include "attn.h"\n#include <stdio.h>\n'
+                   "int main(void) {\n  void* fns[] = {\n" +
+                   "".join(f"    (void*)&{n},\n" for n in names) +
+                   "  };\n  printf(\"%d\\n\", (int)(sizeof fns / sizeof fns[0]));\n"
+                   "  return 0;\n}\n")
+    lib_dir = os.path.dirname(eta.LIB_PATH)
+    res = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                          "-Wno-pedantic", "-I", os.path.join(ROOT, "include"), str(src),
+                          "-L", lib_dir, "-lattn", "-o", str(tmp_path / "abi")],
+                         capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
