@@ -213,3 +213,8 @@ def test_header_is_plain_c_and_links(tmp_path, clib):
                           "-L", lib_dir, "-lattn", "-o", str(tmp_path / "abi")],
                          capture_output=True, text=True)
     assert res.returncode == 0, res.stderr
+
+
+def test_last_cuda_error_starts_clear(clib):
+    # No CUDA call has failed on this thread through the library's launch paths.
+    assert clib.attn_last_cuda_error() == 0
