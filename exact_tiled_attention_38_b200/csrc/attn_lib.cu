@@ -594,14 +594,15 @@ const char* attn_strerror(int code) {
       return "invalid argument (null or misaligned pointer, bad size, Hq % Hkv != 0, or scale "
              "not finite and > 0)";
     case ATTN_ERR_UNSUPPORTED:
-      return "unsupported (head dim not 64 or 128, or device is not sm_100)";
+      return "unsupported (head dim not a multiple of 8 in [8, 256]; decode with d = 64 or 128 "
+             "and B > 65,535; or a device other than sm_100)";
     case ATTN_ERR_CUDA:
       return "CUDA runtime error";
     case ATTN_ERR_TIMEOUT:
       return "a device-side wait gave up; outputs of that launch are undefined";
     case ATTN_ERR_SCRATCH:
-      return "B * Hq * (d + 1) exceeds the fixed scratch of attn_decode_noalloc "
-             "(2,097,152 floats)";
+      return "attn_decode_noalloc: one split-KV partial (B * Hq * (d + 1) floats) exceeds its "
+             "fixed scratch of 2,097,152 floats";
     default:
       return "unknown error code";
   }
@@ -704,18 +705,49 @@ static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 // On the host, g_noalloc_scratch names a host-side stand-in, not device
 // memory: a kernel handed that name would fault or, where the GPU can reach
 // host memory, silently use the wrong memory. The device address is looked up
-// here, once per device, with that device current.
+// here with the device current, once per device and context: the context's
+// unique id is remembered with the address, so after cudaDeviceReset (which
+// ends the context and the module with it) the next call looks the address up
+// again instead of using a dead one.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(ptr);
+}
+
+// Unique id of the calling thread's current context; 0 if there is none.
+unsigned long long current_context_id() {
+  static const CtxGetCurrentFn get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (get_ctx == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 int noalloc_scratch(float** out) {
   static std::mutex mu;
   static float* addr[64] = {};
+  static unsigned long long ctx_id[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  const unsigned long long id = current_context_id();
+  if (addr[dev] == nullptr || id == 0 || id != ctx_id[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return ATTN_ERR_CUDA;
     addr[dev] = static_cast<float*>(p);
+    ctx_id[dev] = current_context_id();  // the look-up made the context current if it was not
   }
   *out = addr[dev];
   return ATTN_OK;
@@ -740,16 +772,9 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
     if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
     return decode_generic<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, 0, st);
   }
-  // One split needs B * Hq * (d + 1) floats; fewer splits are used when the
-  // usual count does not fit, and sizes where even one does not fit are refused.
-  const size_t rows = static_cast<size_t>(B) * Hq;
-  const size_t per_split = rows * (d + 1);
-  if (per_split > kNoAllocScratchFloats) return ATTN_ERR_SCRATCH;
   DeviceInfo info;
   if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
   if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
-  float* scratch = nullptr;
-  if (noalloc_scratch(&scratch) != ATTN_OK) return ATTN_ERR_CUDA;
 
   decode::DParams p;
   p.q = q;
@@ -762,18 +787,35 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
   p.G = Hq / Hkv;
   const int GP = decode_group_tile(p.G);
   p.nchunk = (p.G + GP - 1) / GP;
+  // One split needs B * Hq * (d + 1) floats of scratch; fewer splits than
+  // attn_decode's count are used when that count does not fit. The
+  // tensor-core pass with a single split writes o and lse itself and needs no
+  // scratch, so it runs even when not one split fits; every other case where
+  // not one split fits is refused.
+  const size_t rows = static_cast<size_t>(B) * Hq;
+  const size_t per_split = rows * (d + 1);
   const size_t fit = kNoAllocScratchFloats / per_split;
   const int want = decode_splits(B, Hq, Hkv, d, info.sm_count);
+  const bool tc = decode_use_tc(p.G, d);
   p.nsplit = static_cast<int>(fit < static_cast<size_t>(want) ? fit : want);
+  if (p.nsplit < 1) {
+    if (!tc) return ATTN_ERR_SCRATCH;
+    p.nsplit = 1;
+  }
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
   p.window = 0;
   p.o = nullptr;
   p.lse = nullptr;
-  if (decode_use_tc(p.G, d) && p.nsplit == 1) {  // writes the result directly
+  if (tc && p.nsplit == 1) {  // writes the result directly; no scratch
     p.o = o;
     p.lse = lse;
+    p.part_o = nullptr;
+    p.part_lse = nullptr;
+    return decode_launch_all<128, T>(p, o, lse, st);
   }
+  float* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != ATTN_OK) return ATTN_ERR_CUDA;
   // Every partial slot is written by the split pass before the combine reads
   // it, so nothing in the scratch has to start at zero.
   p.part_o = scratch;

@@ -61,7 +61,8 @@ typedef struct CUstream_st* attn_stream_t;
 enum attn_status {
   ATTN_OK = 0,
   ATTN_ERR_INVALID = -1,     /* null pointer, bad size, misaligned, Hq % Hkv != 0, bad scale */
-  ATTN_ERR_UNSUPPORTED = -2, /* d not a multiple of 8 in [8, 256], or the device is not sm_100 */
+  ATTN_ERR_UNSUPPORTED = -2, /* d not a multiple of 8 in [8, 256]; decode with d = 64 / 128 and
+                                B > 65,535; or the device is not sm_100 */
   ATTN_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
   ATTN_ERR_TIMEOUT = -4,     /* a device-side wait gave up (see attn_get_device_status) */
   ATTN_ERR_SCRATCH = -5      /* attn_decode_noalloc: sizes exceed its fixed scratch */
@@ -139,10 +140,16 @@ int attn_decode_f16(const void* q, const void* kcache, const void* vcache,
  *     allocating library routine.
  *   - One split needs B * Hq * (d + 1) floats. When the usual split count does
  *     not fit, fewer splits are used (results then agree with attn_decode to
- *     rounding); when even one split does not fit, the call returns
- *     ATTN_ERR_SCRATCH and enqueues nothing.
+ *     rounding). When not even one split fits: with d = 128 and 8 to 32 query
+ *     heads per KV head the tensor-core pass runs with one split and writes o
+ *     and lse itself, using no scratch; any other such call returns
+ *     ATTN_ERR_SCRATCH and enqueues nothing. Head sizes other than 64 and 128
+ *     never use the scratch.
  *   - The first call on a device looks up the array's device address (a
- *     runtime call); make that first call before any stream capture.
+ *     runtime call); make that first call before any stream capture. The
+ *     address is remembered with the id of the device's context; after
+ *     cudaDeviceReset (a new context) the next call looks it up again, so
+ *     make the first call after a reset before any capture too.
  *   - Every call on a device uses the same array, which keeps the previous
  *     call's contents (nothing in it needs to start at zero). Calls that can
  *     overlap on the GPU (different streams without ordering between them)

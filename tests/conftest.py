@@ -28,3 +28,20 @@ def lib():
 
     eta.load_library()
     return eta
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print every GPU-vs-oracle comparison of the session: its max errors and
+    how many outputs passed under the one-ulp allowance of `parity.py`."""
+    try:
+        import parity
+    except Exception:  # pragma: no cover
+        return
+    lines = parity.summary_lines()
+    if not lines:
+        return
+    n_allow = sum(r["n_ulp_allowance"] for _, r in parity.RECORDS)
+    terminalreporter.section(f"parity against the fp64 oracle ({len(lines)} comparisons, "
+                             f"{n_allow} outputs under the one-ulp allowance)")
+    for line in lines:
+        terminalreporter.write_line(line)

@@ -61,6 +61,17 @@ def test_strerror_covers_codes(clib):
         assert s and len(s) > 1
 
 
+def test_strerror_messages_state_the_real_limits(clib):
+    msg = lambda c: clib.attn_strerror(c).decode()  # noqa: E731
+    unsup = msg(eta.ATTN_ERR_UNSUPPORTED)
+    # head sizes: any multiple of 8 in [8, 256] is supported (not just 64 / 128)
+    assert "multiple of 8 in [8, 256]" in unsup and "not 64 or 128" not in unsup
+    assert "65,535" in unsup and "sm_100" in unsup
+    scr = msg(eta.ATTN_ERR_SCRATCH)
+    assert "attn_decode_noalloc" in scr and "2,097,152" in scr
+    assert msg(12345) == "unknown error code"
+
+
 # Calls that the host rejects (or finds empty) before touching CUDA.
 FAKE = ctypes.c_void_p(0x10000)
 

@@ -80,7 +80,7 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
         steps, warmup, gpus = 1, 3, 2
 
     called = []
-    monkeypatch.setattr(bench, "cpu_inputs", lambda: called.append(1))
+    monkeypatch.setattr(bench, "headline_head_inputs", lambda: called.append(1))
     assert bench.run_reference(A, 2, 1) == 0   # rank 1: exits without work
     assert called == []
 

@@ -16,8 +16,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
-from parity import TOL_LSE, TOL_O
+from parity import TOL_LSE, TOL_O, compare
 
 pytestmark = pytest.mark.gpu
 
@@ -58,8 +59,56 @@ def test_noalloc_after_a_larger_call_and_with_empty_sequences(lib):
     _call_pair(lib, q, kc, vc, sl, 2)
 
 
+def _oracle_sample(q, kc, vc, sl, Hkv, o, lse, seqs, what):
+    """Compare sequences `seqs` of a no-alloc result with the fp64 oracle."""
+    lens = sl.cpu().tolist()
+    offs = np.concatenate([[0], np.cumsum(lens)])
+    d = q.shape[-1]
+    per = Hkv * d
+    qc, kcc, vcc = q.cpu(), kc.cpu(), vc.cpu()
+    for b in seqs:
+        a, e = int(offs[b]) * per, int(offs[b + 1]) * per
+        o_ref, l_ref = oracle.decode_ref(qc[b:b + 1], kcc[a:e], vcc[a:e], sl.cpu()[b:b + 1],
+                                         d ** -0.5, Hkv)
+        compare(o[b:b + 1], lse[b:b + 1], o_ref, l_ref, torch.bfloat16, f"{what} seq {b}")
+
+
+def test_noalloc_fewer_splits_than_usual(lib):
+    # One split of B=128, Hq=32, d=128 needs 528,384 floats: 3 fit in the
+    # scratch, while attn_decode uses 4 splits here on a 148-SM B200.
+    B, Hq, Hkv, d = 128, 32, 8, 128
+    per_split = B * Hq * (d + 1)
+    fit = 2_097_152 // per_split
+    want = lib.attn_decode_num_splits(B, Hq, Hkv, d)
+    assert fit == 3 and want > fit, (fit, want)
+    sl = workloads.decode_seqlens(B, 1, 3000, 47)
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, d, sl, torch.bfloat16, seed=47,
+                                            device=DEV)
+    _call_pair(lib, q, kc, vc, sl, Hkv)
+    o, lse = lib.attn_decode_noalloc(q, kc, vc, sl, Hkv=Hkv)
+    torch.cuda.synchronize()
+    _oracle_sample(q, kc, vc, sl, Hkv, o, lse, range(0, B, 9), "noalloc 3 of 4 splits")
+
+
+def test_noalloc_tensor_core_single_split_beyond_scratch(lib):
+    # Groups of 8..32 heads at d = 128 with one split per sequence need no
+    # scratch: even sizes where one split would not fit the array run (this one
+    # needs 4096 * 32 * 129 floats per split, about 8 times the array).
+    B, Hq, Hkv, d = 4096, 32, 4, 128
+    assert B * Hq * (d + 1) > 2_097_152
+    assert lib.attn_decode_num_splits(B, Hq, Hkv, d) == 1
+    sl = workloads.decode_seqlens(B, 0, 48, 53)
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, d, sl, torch.bfloat16, seed=53,
+                                            device=DEV)
+    _call_pair(lib, q, kc, vc, sl, Hkv)
+    o, lse = lib.attn_decode_noalloc(q, kc, vc, sl, Hkv=Hkv)
+    torch.cuda.synchronize()
+    _oracle_sample(q, kc, vc, sl, Hkv, o, lse, range(0, B, 61), "noalloc tensor-core B=4096")
+
+
 def test_noalloc_refuses_sizes_beyond_its_scratch(lib):
-    # B * Hq * (d + 1) floats per split; 16384 * 8 * 129 is above 2,097,152.
+    # B * Hq * (d + 1) floats per split on the CUDA-core pass (4 query heads
+    # per KV head); 16384 * 8 * 129 is above 2,097,152.
     B, Hq, Hkv, d = 16384, 8, 2, 128
     q = torch.zeros(B, Hq, d, device=DEV, dtype=torch.bfloat16)
     kc = torch.zeros(64, device=DEV, dtype=torch.bfloat16)
