@@ -233,6 +233,20 @@ class ClockSampler:
         return out
 
 
+def merged_clocks(samplers):
+    """One clock record over several sampled regions (median of all samples)."""
+    sm = [x for c in samplers for x in c.sm]
+    reasons = sorted(set().union(*(c.reasons for c in samplers))) if samplers else []
+    out = {"sm_mhz": statistics.median(sm) if sm else None,
+           "sm_max_mhz": samplers[0].max_sm if samplers else None, "reasons": reasons,
+           "samples": len(sm), "source": "nvml",
+           "per_phase": [c.summary() for c in samplers]}
+    errs = [c.error for c in samplers if c.error]
+    if errs:
+        out["error"] = errs[0]
+    return out
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def blas_threads() -> int:
     try:
@@ -494,54 +508,66 @@ def run_ours(args, world, rank, local):
         flush_rd.max()
 
     n_ev = len(PREFILLS) + 1
+    kernel_names = [PREFILL_KEYS[w.name] for w, *_ in pre] + ["decode"]
 
-    def step(evs=None):
-        for i, (w, q, k, v, o, lse) in enumerate(pre):
-            flush_l2()
-            if evs:
-                evs[2 * i].record(stream)
-            eta.attn_fwd(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal, stream=stream)
-            if evs:
-                evs[2 * i + 1].record(stream)
-        flush_l2()
-        if evs:
-            evs[2 * n_ev - 2].record(stream)
-        eta.attn_decode(dq, dkc, dvc, dsl, DECODE.Hkv, o=do, lse=dlse, scale=DECODE.scale,
-                        stream=stream)
-        if evs:
-            evs[2 * n_ev - 1].record(stream)
+    def launch(name):
+        if name == "decode":
+            eta.attn_decode(dq, dkc, dvc, dsl, DECODE.Hkv, o=do, lse=dlse, scale=DECODE.scale,
+                            stream=stream)
+            return
+        w, q, k, v, o, lse = pre[kernel_names.index(name)]
+        eta.attn_fwd(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal, stream=stream)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    code, raw = eta.attn_get_device_status(stream)
-    if code != eta.ATTN_OK:
-        raise RuntimeError(f"device status {code} ({raw:#x}) after warm-up")
+    # The step's kernels are timed in phases, shortest first: a launch of
+    # about 0.13 s (the 128K prefill) holds the GPU at its power-capped clock
+    # for a while afterwards, which would slow the short kernels that follow
+    # it. Each phase has its own warm-up and clock record; a step is one pass
+    # of every phase's kernels over their batch, so ms_per_step is the sum of
+    # the phases' per-step times.
+    phases = [("decode", "2k"), ("32k",), ("128k",)]
+    ms, phase_ms, phase_clocks = {}, {}, {}
+    for names in phases:
+        def step(evs=None):
+            for i, name in enumerate(names):
+                flush_l2()
+                if evs:
+                    evs[2 * i].record(stream)
+                launch(name)
+                if evs:
+                    evs[2 * i + 1].record(stream)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_ev)]
-           for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        t_end.record(stream)
+        for _ in range(args.warmup):
+            step()
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    code, raw = eta.attn_get_device_status(stream)
-    if code != eta.ATTN_OK:
-        raise RuntimeError(f"device status {code} ({raw:#x}) in the timed loop")
-
-    ms = [sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs) / args.steps
-          for i in range(n_ev)]
-    step_ms = t_start.elapsed_time(t_end) / args.steps
-    ms_max = reduce_max(ms + [step_ms])
-    step_ms_max = ms_max.pop()
+        code, raw = eta.attn_get_device_status(stream)
+        if code != eta.ATTN_OK:
+            raise RuntimeError(f"device status {code} ({raw:#x}) after warm-up of {names}")
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]
+               for _ in range(args.steps)]
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clocks:
+            t_start.record(stream)
+            for i in range(args.steps):
+                step(evs[i])
+            t_end.record(stream)
+            torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        code, raw = eta.attn_get_device_status(stream)
+        if code != eta.ATTN_OK:
+            raise RuntimeError(f"device status {code} ({raw:#x}) in the timed loop of {names}")
+        for i, name in enumerate(names):
+            ms[name] = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs) / args.steps
+        phase_ms["+".join(names)] = t_start.elapsed_time(t_end) / args.steps
+        phase_clocks["+".join(names)] = clocks
+    order = kernel_names + list(phase_ms)
+    red = reduce_max([ms[n] for n in kernel_names] + [phase_ms[n] for n in phase_ms])
+    ms_max = dict(zip(order, red))
+    step_ms_max = sum(ms_max[n] for n in phase_ms)
 
     # ---- end to end through the public API, host buffers in pinned memory:
     # every step copies each workload's inputs host -> device, runs the call
@@ -598,19 +624,22 @@ def run_ours(args, world, rank, local):
     peaks, src = load_peaks()
     kv_bytes = decode_kv_bytes(sl_cpu.numpy(), DECODE.Hkv, DECODE.d)
     dbytes = decode_bytes(sl_cpu.numpy(), DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.d)
-    dec_ms = ms[-1]
+    dec_ms = ms["decode"]
     dec_ach = dbytes / (dec_ms * 1e-3) / 1e9
     hl_flops = prefill_flops(HEADLINE)
-    value = aggregate_throughput(hl_flops, world, ms_max[0]) / 1e12
+    value = aggregate_throughput(hl_flops, world, ms_max["128k"]) / 1e12
     # The 128K launch (about 0.13 s, most of a step's time) runs long enough to
     # sit at the power-capped clock: its fraction is taken of the sustained
     # measured rate, the shorter launches' of the burst rate; both are given.
-    rl = {PREFILL_KEYS[w.name]: prefill_roofline(w, ms[i], peaks, src,
+    rl = {PREFILL_KEYS[w.name]: prefill_roofline(w, ms[PREFILL_KEYS[w.name]], peaks, src,
                                                  "sustained" if w is HEADLINE else "burst")
-          for i, (w, *_) in enumerate(pre)}
+          for w, *_ in pre}
     prefill_lines = {PREFILL_KEYS[w.name]: {
-        "value": aggregate_throughput(prefill_flops(w), world, ms_max[i]) / 1e12,
-        "unit": "TFLOP/s", "ms_per_launch": ms[i]} for i, (w, *_) in enumerate(pre)}
+        "value": aggregate_throughput(prefill_flops(w), world, ms_max[PREFILL_KEYS[w.name]]) / 1e12,
+        "unit": "TFLOP/s", "ms_per_launch": ms[PREFILL_KEYS[w.name]],
+        "clocks": phase_clocks[next(n for n in phase_clocks
+                                    if PREFILL_KEYS[w.name] in n.split("+"))].summary()}
+        for w, *_ in pre}
     e2e_seg = {PREFILL_KEYS[w.name]: {
         "value": aggregate_throughput(prefill_flops(w), world, e2e_ms[i]) / 1e12,
         "unit": "TFLOP/s", "h2d_bytes": seg_h2d[i], "d2h_bytes": seg_d2h[i]}
@@ -631,8 +660,10 @@ def run_ours(args, world, rank, local):
                        "d": DECODE.d, "kv_tokens": int(sl_cpu.sum()), "kv_bytes": kv_bytes,
                        "nsplit": eta.attn_decode_num_splits(DECODE.B, DECODE.Hq, DECODE.Hkv,
                                                             DECODE.d)},
-            "step": "prefill 128K, prefill 32K, prefill 2K, decode; each kernel timed alone "
-                    "with CUDA events on its stream",
+            "step": "decode and prefill 2K, then prefill 32K, then prefill 128K, each in its "
+                    "own timed phase of `steps` iterations (shortest first, so that the 128K "
+                    "launches' power-capped clock does not carry over into the short kernels); "
+                    "each kernel timed with CUDA events on its stream",
             "l2": "flushed before every kernel (256 MiB write, then a 256 MiB read that "
                   "evicts its dirty lines; outside the kernel events); the 128K and 32K "
                   "inputs and the decode cache are also larger than L2",
@@ -656,14 +687,16 @@ def run_ours(args, world, rank, local):
             "nominal": {"peak": NOMINAL_PEAKS["hbm_gbs"],
                         "frac": dec_ach / NOMINAL_PEAKS["hbm_gbs"]}},
         "prefill": prefill_lines,
-        "decode": {"value": aggregate_throughput(kv_bytes, world, ms_max[-1]) / 1e9,
-                   "unit": "GB/s (KV cache read)", "ms_per_call": dec_ms},
+        "decode": {"value": aggregate_throughput(kv_bytes, world, ms_max["decode"]) / 1e9,
+                   "unit": "GB/s (KV cache read)", "ms_per_call": dec_ms,
+                   "clocks": phase_clocks["decode+2k"].summary()},
         "e2e": {"value": e2e_seg["128k"]["value"], "unit": "TFLOP/s",
                 "h2d_bytes_per_step": seg_h2d[0], "d2h_bytes_per_step": seg_d2h[0],
                 "what": "the 128K prefill through the public binding: H2D of q, k, v from "
                         "pinned host memory, attn_fwd, D2H of O and LSE, per step",
                 "segments": e2e_seg, "steps": e2e_steps},
-        "clocks": clocks.summary(),
+        "clocks": merged_clocks(list(phase_clocks.values())),
+        "phases_ms_per_step": phase_ms,
         # 3 prefill launches + decode split pass + combine per step
         "gpu_launches": (len(PREFILLS) + 2) * args.steps,
     }
