@@ -470,9 +470,27 @@ def run_ours(args, world, rank, local):
     # library's pool. A materialised fp32 score matrix would take
     # B * Hq * Nq * Nk * 4 bytes.
     eta.attn_get_device_status(stream)  # loads the library's module (code, static arrays)
-    pre = []  # per prefill workload: (w, q, k, v, o, lse)
     memory = {"how": "device-wide free memory before and after the first call"}
-    for w in PREFILLS:
+    data = {}  # kernel name -> its inputs and outputs, set up when its phase starts
+
+    def setup(name):
+        torch.cuda.synchronize()
+        if name == "decode":
+            sl_cpu = workloads.decode_seqlens(DECODE.B, DECODE.lmin, DECODE.lmax,
+                                              DECODE.seed + seed_off)
+            dq, dkc, dvc, dsl = workloads.decode_inputs(DECODE, device=dev, seqlens=sl_cpu,
+                                                        seed=DECODE.seed + seed_off)
+            do = torch.empty_like(dq)
+            dlse = torch.empty(DECODE.B, DECODE.Hq, device=dev, dtype=torch.float32)
+            torch.cuda.synchronize()
+            free0 = torch.cuda.mem_get_info(dev)[0]
+            eta.attn_decode(dq, dkc, dvc, dsl, DECODE.Hkv, o=do, lse=dlse, scale=DECODE.scale,
+                            stream=stream)
+            torch.cuda.synchronize()
+            memory["decode_library_bytes"] = free0 - torch.cuda.mem_get_info(dev)[0]
+            data[name] = (sl_cpu, dq, dkc, dvc, dsl, do, dlse)
+            return
+        w = next(x for x in PREFILLS if PREFILL_KEYS[x.name] == name)
         q, k, v = workloads.prefill_inputs(w, device=dev, seed=w.seed + seed_off)
         o = torch.empty_like(q)
         lse = torch.empty(w.B, w.Hq, w.Nq, device=dev, dtype=torch.float32)
@@ -480,22 +498,9 @@ def run_ours(args, world, rank, local):
         free0 = torch.cuda.mem_get_info(dev)[0]
         eta.attn_fwd(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal, stream=stream)
         torch.cuda.synchronize()
-        memory[f"prefill_{PREFILL_KEYS[w.name]}_library_bytes"] = free0 - torch.cuda.mem_get_info(dev)[0]
-        memory[f"prefill_{PREFILL_KEYS[w.name]}_score_matrix_fp32_bytes"] = (
-            w.B * w.Hq * w.Nq * w.Nk * 4)
-        pre.append((w, q, k, v, o, lse))
-    sl_cpu = workloads.decode_seqlens(DECODE.B, DECODE.lmin, DECODE.lmax,
-                                      DECODE.seed + seed_off)
-    dq, dkc, dvc, dsl = workloads.decode_inputs(DECODE, device=dev, seqlens=sl_cpu,
-                                                seed=DECODE.seed + seed_off)
-    do = torch.empty_like(dq)
-    dlse = torch.empty(DECODE.B, DECODE.Hq, device=dev, dtype=torch.float32)
-    torch.cuda.synchronize()
-    free0 = torch.cuda.mem_get_info(dev)[0]
-    eta.attn_decode(dq, dkc, dvc, dsl, DECODE.Hkv, o=do, lse=dlse, scale=DECODE.scale,
-                    stream=stream)
-    torch.cuda.synchronize()
-    memory["decode_library_bytes"] = free0 - torch.cuda.mem_get_info(dev)[0]
+        memory[f"prefill_{name}_library_bytes"] = free0 - torch.cuda.mem_get_info(dev)[0]
+        memory[f"prefill_{name}_score_matrix_fp32_bytes"] = w.B * w.Hq * w.Nq * w.Nk * 4
+        data[name] = (w, q, k, v, o, lse)
 
     # L2 flush before every kernel: write 256 MiB (> 126 MB L2), then read
     # another 256 MiB so that the dirty lines of the write are evicted (written
@@ -507,26 +512,30 @@ def run_ours(args, world, rank, local):
         flush.zero_()
         flush_rd.max()
 
-    n_ev = len(PREFILLS) + 1
-    kernel_names = [PREFILL_KEYS[w.name] for w, *_ in pre] + ["decode"]
+    kernel_names = [PREFILL_KEYS[w.name] for w in PREFILLS] + ["decode"]
 
     def launch(name):
         if name == "decode":
+            _, dq, dkc, dvc, dsl, do, dlse = data[name]
             eta.attn_decode(dq, dkc, dvc, dsl, DECODE.Hkv, o=do, lse=dlse, scale=DECODE.scale,
                             stream=stream)
             return
-        w, q, k, v, o, lse = pre[kernel_names.index(name)]
+        w, q, k, v, o, lse = data[name]
         eta.attn_fwd(q, k, v, o=o, lse=lse, scale=w.scale, causal=w.causal, stream=stream)
 
-    # The step's kernels are timed in phases, shortest first: a launch of
-    # about 0.13 s (the 128K prefill) holds the GPU at its power-capped clock
-    # for a while afterwards, which would slow the short kernels that follow
-    # it. Each phase has its own warm-up and clock record; a step is one pass
-    # of every phase's kernels over their batch, so ms_per_step is the sum of
-    # the phases' per-step times.
+    # The step's kernels are timed in phases, shortest first, and each phase
+    # sets up its own workloads just before it: a launch of about 0.13 s (the
+    # 128K prefill) holds the GPU at its power-capped clock for a while
+    # afterwards, which would slow the short kernels if they followed it. Each
+    # phase has its own warm-up and clock record (the short phase sampled
+    # every millisecond); a step is one pass of every phase's kernels over
+    # their batch, so ms_per_step is the sum of the phases' per-step times.
     phases = [("decode", "2k"), ("32k",), ("128k",)]
     ms, phase_ms, phase_clocks = {}, {}, {}
     for names in phases:
+        for name in names:
+            setup(name)
+
         def step(evs=None):
             for i, name in enumerate(names):
                 flush_l2()
@@ -549,7 +558,8 @@ def run_ours(args, world, rank, local):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        with ClockSampler(local) as clocks:
+        period = 0.001 if names == phases[0] else 0.005
+        with ClockSampler(local, period_s=period) as clocks:
             t_start.record(stream)
             for i in range(args.steps):
                 step(evs[i])
@@ -564,6 +574,9 @@ def run_ours(args, world, rank, local):
             ms[name] = sum(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs) / args.steps
         phase_ms["+".join(names)] = t_start.elapsed_time(t_end) / args.steps
         phase_clocks["+".join(names)] = clocks
+    pre = [data[PREFILL_KEYS[w.name]] for w in PREFILLS]
+    n_ev = len(PREFILLS) + 1
+    sl_cpu, dq, dkc, dvc, dsl, do, dlse = data["decode"]
     order = kernel_names + list(phase_ms)
     red = reduce_max([ms[n] for n in kernel_names] + [phase_ms[n] for n in phase_ms])
     ms_max = dict(zip(order, red))

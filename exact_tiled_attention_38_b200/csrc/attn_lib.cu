@@ -4,7 +4,10 @@
 //   prefill_sm100.cuh    prefill, d = 64 / 128 (tcgen05, TMA)
 //   decode_sm100.cuh     decode split pass on CUDA cores (d = 64, groups <= 4)
 //                        and the LSE combine
-//   decode_tc_sm100.cuh  decode split pass on tcgen05 (d = 128, groups 8..32)
+//   decode_ps_sm100.cuh  decode as one persistent streaming pass on tcgen05
+//                        (d = 128, groups 8..32): plan, stream, gather
+//   decode_tc_sm100.cuh  helpers of the tcgen05 decode (and its earlier
+//                        one-CTA-per-split pass, kept as a knob)
 //   generic_fwd.cuh      prefill and decode for the other head sizes
 //   merge.cuh            LSE merge of partial results (context parallelism)
 #include <cuda.h>
@@ -16,6 +19,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "decode_ps_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "decode_tc_sm100.cuh"
 #include "generic_fwd.cuh"
@@ -348,8 +352,48 @@ inline int decode_group_tile(int G) { return (G <= 4 || ETA_DECODE_MAX_GP == 4) 
 #ifndef ETA_DECODE_TC_WAVES
 #define ETA_DECODE_TC_WAVES 2
 #endif
+// Persistent streaming pass (decode_ps_sm100.cuh) for d = 128 and
+// ETA_DECODE_PS_MIN_G to 32 query heads per KV head; 0 turns it off (the
+// one-CTA-per-split tensor-core pass then takes groups of 8 to 32). Measured
+// on B200 (64 sequences of 1K-8K tokens, d = 128, median of 30 launches, L2
+// flushed): group 4 0.236 ms against 0.246 ms on the CUDA-core pass, group 8
+// 0.238 / 0.248 ms and group 16 0.240 / 0.256 ms against the one-CTA-per-split
+// tensor-core pass, MQA 0.088 / 0.099 ms; a single head per KV head (MHA)
+// 0.236 ms against 0.232 ms on the CUDA-core pass, which keeps it.
+#ifndef ETA_DECODE_PS_MIN_G
+#define ETA_DECODE_PS_MIN_G 2
+#endif
+inline bool decode_use_ps(int G, int d) {
+  return ETA_DECODE_PS_MIN_G > 0 && d == 128 && G >= ETA_DECODE_PS_MIN_G && G <= 32;
+}
 inline bool decode_use_tc(int G, int d) {
-  return d == 128 && G >= ETA_DECODE_TC_MIN_G && G <= 32;
+  return !decode_use_ps(G, d) && d == 128 && G >= ETA_DECODE_TC_MIN_G && G <= 32;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Device workspace of the persistent pass, byte offsets: the plan (token
+// offsets int64 [B], tile offsets int32 [B + 1]) and, when CTAs take equal
+// tile ranges, the partials of segments cut between CTAs (slot segment + cta:
+// B * Hkv + nc - 1 slots of G rows).
+struct PsLayout {
+  size_t tok_off, tile_off, part_o, part_lse, total;
+};
+inline PsLayout ps_layout(int B, int Hkv, int G, int nc, bool partials) {
+  PsLayout L;
+  L.tok_off = 0;
+  L.tile_off = align_up(static_cast<size_t>(B) * 8, 256);
+  size_t end = L.tile_off + (static_cast<size_t>(B) + 1) * 4;
+  L.part_o = L.part_lse = 0;
+  if (partials) {
+    const size_t slots = static_cast<size_t>(B) * Hkv + nc - 1;
+    L.part_o = align_up(end, 256);
+    end = L.part_o + slots * G * decode_ps::D * 4;
+    L.part_lse = align_up(end, 256);
+    end = L.part_lse + slots * G * 4;
+  }
+  L.total = align_up(end, 256);
+  return L;
 }
 
 int decode_splits(int B, int Hq, int Hkv, int d, int sm_count) {
@@ -399,6 +443,71 @@ int launch_decode_tc(const decode::DParams& p, cudaStream_t st) {
                   static_cast<unsigned>(p.B));
   kern<<<grid, decode_tc::kThreads, smem, st>>>(p);
   return launch_status();
+}
+
+// Plan, persistent stream and gather of the d = 128 decode; `ws` holds the
+// layout `L`. seg_aligned: whole segments per CTA (L has no partials).
+template <int NP, typename T>
+int launch_decode_ps(const CUtensorMap& tq, decode_ps::PParams p, const PsLayout& L, char* ws,
+                     int nc, cudaStream_t st) {
+  auto kern = decode_ps::attn_decode_persistent_kernel<NP, T>;
+  constexpr int smem = decode_ps::PCfg<NP>::kSmemBytes;
+  static PerDeviceOnce attr;
+  const cudaError_t attr_err = attr.run([&]() {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err);
+  long long* tok_off = reinterpret_cast<long long*>(ws + L.tok_off);
+  int* tile_off = reinterpret_cast<int*>(ws + L.tile_off);
+  p.tok_off = tok_off;
+  p.tile_off = tile_off;
+  p.part_o = L.part_o ? reinterpret_cast<float*>(ws + L.part_o) : nullptr;
+  p.part_lse = L.part_lse ? reinterpret_cast<float*>(ws + L.part_lse) : nullptr;
+  decode_ps::attn_decode_plan_kernel<<<1, decode_ps::kPlanThreads, 0, st>>>(
+      p.seqlens, tok_off, tile_off, p.B, p.Hkv, p.window);
+  int rc = launch_status();
+  if (rc != ATTN_OK) return rc;
+  kern<<<nc, decode_ps::kThreads, smem, st>>>(tq, p);
+  rc = launch_status();
+  if (rc != ATTN_OK) return rc;
+  const long long rows = static_cast<long long>(p.B) * p.Hq;
+  decode_ps::attn_decode_gather_kernel<T>
+      <<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(p, nc);
+  return launch_status();
+}
+
+// The persistent decode for d = 128: q's tensor map (rows of the G heads of
+// one KV head, box padded to NP rows), then the three kernels. `ws` must hold
+// ps_layout(B, Hkv, G, nc, !seg_aligned).
+template <typename T>
+int decode_ps_run(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* o,
+                  float* lse, int B, int Hq, int Hkv, float scale, int window, char* ws,
+                  bool seg_aligned, int nc, cudaStream_t st) {
+  constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+  const int G = Hq / Hkv;
+  const int NP = G <= 16 ? 16 : 32;
+  CUtensorMap tq;
+  const int rc = encode_3d(&tq, q, bf16, decode_ps::D, G, static_cast<long long>(B) * Hkv,
+                           static_cast<unsigned>(NP));
+  if (rc != ATTN_OK) return rc;
+  decode_ps::PParams p;
+  p.q = q;
+  p.kc = kc;
+  p.vc = vc;
+  p.seqlens = seqlens;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.window = window;
+  p.seg_aligned = seg_aligned ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_ns = kDefaultWaitNs;
+  const PsLayout L = ps_layout(B, Hkv, G, nc, !seg_aligned);
+  return NP == 16 ? launch_decode_ps<16, T>(tq, p, L, ws, nc, st)
+                  : launch_decode_ps<32, T>(tq, p, L, ws, nc, st);
 }
 
 template <int D, typename T>
@@ -472,6 +581,19 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
   if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
   if (!tensor_core_d(d))
     return decode_generic<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, window, st);
+  if (decode_use_ps(Hq / Hkv, d)) {
+    const int nc = info.sm_count;
+    const PsLayout L = ps_layout(B, Hkv, Hq / Hkv, nc, true);
+    void* ws = nullptr;
+    cudaMemPool_t pool;
+    if (workspace_pool(&pool) != ATTN_OK) return ATTN_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(&ws, L.total, pool, st) != cudaSuccess) return ATTN_ERR_CUDA;
+    const int rc = decode_ps_run<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, scale, window,
+                                    static_cast<char*>(ws), false, nc, st);
+    const cudaError_t fe = cudaFreeAsync(ws, st);
+    if (rc != ATTN_OK) return rc;
+    return fe == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
 
   decode::DParams p;
   p.q = q;
@@ -581,6 +703,7 @@ int attn_decode_f16(const void* q, const void* kcache, const void* vcache,
 int attn_decode_num_splits(int B, int Hq, int Hkv, int d) {
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID;
   if (!eta::api::tensor_core_d(d)) return eta::api::generic_d(d) ? 1 : ATTN_ERR_UNSUPPORTED;
+  if (eta::api::decode_use_ps(Hq / Hkv, d)) return 1;  // one streaming pass, no fixed split
   eta::api::DeviceInfo info;
   if (eta::api::device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
   return eta::api::decode_splits(B, Hq, Hkv, d, info.sm_count);
@@ -775,6 +898,19 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
   DeviceInfo info;
   if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
   if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
+  if (decode_use_ps(Hq / Hkv, d)) {
+    // The plan always fits (B <= 65,535); the partials of equal tile ranges
+    // when they fit, else every CTA takes whole segments and writes its
+    // results directly.
+    const int nc = info.sm_count;
+    const size_t cap = kNoAllocScratchFloats * sizeof(float);
+    const bool seg_aligned = ps_layout(B, Hkv, Hq / Hkv, nc, true).total > cap;
+    if (ps_layout(B, Hkv, Hq / Hkv, nc, !seg_aligned).total > cap) return ATTN_ERR_SCRATCH;
+    float* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != ATTN_OK) return ATTN_ERR_CUDA;
+    return decode_ps_run<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, scale, 0,
+                            reinterpret_cast<char*>(scratch), seg_aligned, nc, st);
+  }
 
   decode::DParams p;
   p.q = q;

@@ -1,0 +1,679 @@
+// Exact attention, decode, as one persistent streaming pass on the tensor
+// cores (sm_100a), head size 128, up to 32 query heads per KV head.
+//
+// Generating a token re-reads the whole KV cache of its sequence (first page,
+// the token-generation case; zimaspace page, "Reduced IO Is Not the Same as
+// Eliminating KV Cache"), so decode is a stream over the cache and its speed
+// is the rate at which each SM keeps that stream moving. The work is cut into
+// tiles of 128 keys of one (sequence b, KV head g) -- a "segment" -- and the
+// tiles of all segments, in order, are divided into equal contiguous ranges,
+// one per CTA (one CTA per SM). A CTA streams its range without a restart at
+// segment boundaries: the K/V ring, the score products and the running
+// softmax (aikaboom page "11.4d FlashAttention", "Tiling" and "Online
+// Softmax") carry on, and at the end of each piece of a segment the CTA
+// writes either the result itself (the whole segment lay in its range) or a
+// normalised partial with its log-sum-exp, which the gather kernel merges.
+//
+// Three kernels per call:
+//   attn_decode_plan_kernel        one CTA: per sequence, token offset in the
+//                                  packed cache (int64) and tile offset in the
+//                                  global tile order (int32 prefix over
+//                                  sequences, KV heads included)
+//   attn_decode_persistent_kernel  the stream (below)
+//   attn_decode_gather_kernel      one warp per (sequence, query head): merges
+//                                  the partials of segments cut between CTAs,
+//                                  writes O = 0, LSE = -inf for empty ones
+//
+// Per tile (G query heads of KV head g, padded to NP = 16 or 32):
+//   S^T = K_j Q^T      M = 128 keys, N = NP, K = 128 dims; A = K tile
+//                      (K-major), B = Q (K-major); fp32 in tensor memory,
+//                      lane = key, column = head (two buffers)
+//   softmax            warp w owns keys 32w..32w+31; per head the tile max by
+//                      shuffles and across the four warps through shared
+//                      memory; p = 2^(s*c - m) with a lazily moved running max
+//                      per head; P^T [head][key] rounded to the input type in
+//                      shared memory (two buffers); l kept per key slot
+//   O^T += V_j^T P^T   M = 128 dims, N = NP, K = 128 keys; A = the V tile read
+//                      MN-major, B = P^T (K-major); fp32 in tensor memory
+// Q of each segment comes in by TMA (two buffers, the next segment's Q loaded
+// while the current one runs); K and V by 16-byte cp.async straight into the
+// 128-byte-swizzled layout, zero-filled past the segment's last key (the
+// packed cache's extent is only known on the device).
+//
+// Warp roles (256 threads): warps 0-3 softmax and epilogue, warp 4 tensor
+// memory owner, MMA issue and Q loads (whole warp, one elected lane), warps
+// 5-7 producers, each owning one 64 KB ring stage. Every wait is bounded.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <type_traits>
+
+#include "common.cuh"
+#include "decode_tc_sm100.cuh"
+
+namespace eta {
+namespace decode_ps {
+
+constexpr int D = 128;
+constexpr int TK = 128;  // keys per tile
+constexpr int kStages = 3;
+constexpr int kSoftWarps = 4;
+constexpr int kMmaWarp = 4;
+constexpr int kProdWarp0 = 5;
+constexpr int kThreads = 32 * (kProdWarp0 + kStages);
+constexpr float kRescaleThreshold = 8.0f;
+constexpr uint32_t kTmemCols = 128;
+constexpr int kPlanThreads = 1024;
+
+enum : unsigned {
+  kSiteFull = 0x41,
+  kSiteEmpty = 0x42,
+  kSiteS = 0x43,
+  kSiteP = 0x44,
+  kSitePv = 0x45,
+  kSiteX = 0x46,
+  kSiteQ = 0x47,
+  kSiteDrain = 0x48,
+  kSiteQFree = 0x49,
+};
+
+struct PParams {
+  const void* q;
+  const void* kc;
+  const void* vc;
+  const int* seqlens;
+  const long long* tok_off;  // [B]: token offset of sequence b in the packed cache
+  const int* tile_off;       // [B + 1]: first global tile of sequence b (all its KV heads)
+  void* o;                   // [B][Hq][D], input type
+  float* lse;                // [B][Hq] natural log, or NULL
+  float* part_o;             // [slots][G][D]: normalised partial O of a cut segment
+  float* part_lse;           // [slots][G]: its log-sum-exp, log2 units
+  int B;
+  int Hq;
+  int Hkv;
+  int G;
+  int window;       // > 0: each new token reads only the last `window` cached tokens
+  int seg_aligned;  // 1: CTAs take whole segments (no partials); 0: equal tile ranges
+  float scale_log2;
+  uint64_t wait_ns;
+};
+
+// Keys of sequence b read: [first_key, len).
+__device__ __forceinline__ int first_key(int len, int window) {
+  return (window > 0 && len > window) ? len - window : 0;
+}
+
+// ------------------------------------------------------------------ plan
+// Exclusive prefix sums over the B sequences (one CTA): token offsets of the
+// packed cache and tile offsets of the global tile order (Hkv segments of
+// ceil(keys read / 128) tiles per sequence). tile_off[B] is the total.
+__global__ void __launch_bounds__(kPlanThreads) attn_decode_plan_kernel(const int* __restrict__ seqlens,
+                                                                      long long* __restrict__ tok_off,
+                                                                      int* __restrict__ tile_off,
+                                                                      int B, int Hkv, int window) {
+  __shared__ long long s_tok[kPlanThreads / 32];
+  __shared__ long long s_til[kPlanThreads / 32];
+  const int per = (B + kPlanThreads - 1) / kPlanThreads;  // consecutive sequences per thread
+  const int b0 = threadIdx.x * per;
+  const int b1 = min(B, b0 + per);
+  long long tok = 0, til = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int len = max(seqlens[b], 0);
+    tok += len;
+    til += static_cast<long long>(Hkv) * ((len - first_key(len, window) + TK - 1) / TK);
+  }
+  // inclusive scan over the block: warps, then warp totals
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long xt = tok, xl = til;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long yt = __shfl_up_sync(0xffffffffu, xt, o);
+    const long long yl = __shfl_up_sync(0xffffffffu, xl, o);
+    if (lane >= o) {
+      xt += yt;
+      xl += yl;
+    }
+  }
+  if (lane == 31) {
+    s_tok[warp] = xt;
+    s_til[warp] = xl;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    long long wt = s_tok[lane], wl = s_til[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long yt = __shfl_up_sync(0xffffffffu, wt, o);
+      const long long yl = __shfl_up_sync(0xffffffffu, wl, o);
+      if (lane >= o) {
+        wt += yt;
+        wl += yl;
+      }
+    }
+    s_tok[lane] = wt;
+    s_til[lane] = wl;
+  }
+  __syncthreads();
+  long long t_run = xt - tok + (warp > 0 ? s_tok[warp - 1] : 0);  // exclusive
+  long long l_run = xl - til + (warp > 0 ? s_til[warp - 1] : 0);
+  for (int b = b0; b < b1; ++b) {
+    const int len = max(seqlens[b], 0);
+    tok_off[b] = t_run;
+    tile_off[b] = static_cast<int>(l_run);
+    t_run += len;
+    l_run += static_cast<long long>(Hkv) * ((len - first_key(len, window) + TK - 1) / TK);
+  }
+  if (threadIdx.x == kPlanThreads - 1) tile_off[B] = static_cast<int>(s_til[31]);
+}
+
+// Tile range [lo, hi) of CTA c of nc in the global tile order.
+struct Range {
+  long long lo, hi;
+};
+
+__device__ __forceinline__ long long segment_start(const PParams& p, long long s, long long T) {
+  const long long S = static_cast<long long>(p.B) * p.Hkv;
+  if (s >= S) return T;
+  const int b = static_cast<int>(s / p.Hkv);
+  const int g = static_cast<int>(s - static_cast<long long>(b) * p.Hkv);
+  const int nt = (p.tile_off[b + 1] - p.tile_off[b]) / p.Hkv;
+  return p.tile_off[b] + static_cast<long long>(g) * nt;
+}
+
+__device__ __forceinline__ Range cta_range(const PParams& p, int c, int nc) {
+  const long long T = p.tile_off[p.B];
+  Range r;
+  if (p.seg_aligned) {
+    const long long S = static_cast<long long>(p.B) * p.Hkv;
+    r.lo = segment_start(p, c * S / nc, T);
+    r.hi = segment_start(p, (c + 1) * S / nc, T);
+  } else {
+    r.lo = c * T / nc;
+    r.hi = (c + 1) * T / nc;
+  }
+  return r;
+}
+
+// The CTA whose equal tile range holds global tile t (tile-balanced mode).
+__host__ __device__ __forceinline__ int cta_of(long long t, long long T, int nc) {
+  return static_cast<int>(((t + 1) * nc - 1) / T);
+}
+
+// Position of a global tile: sequence b, KV head g, tile i of nt in the segment.
+struct Cursor {
+  int b, g, i, nt;
+  int len, k0;        // keys read of sequence b: [k0, len)
+  long long tok;      // token offset of sequence b
+
+  __device__ __forceinline__ void load_seq(const PParams& p) {
+    nt = (p.tile_off[b + 1] - p.tile_off[b]) / p.Hkv;
+    len = max(p.seqlens[b], 0);
+    k0 = first_key(len, p.window);
+    tok = p.tok_off[b];
+  }
+  __device__ __forceinline__ void seek(const PParams& p, long long t) {
+    int lo = 0, hi = p.B - 1;  // largest b with tile_off[b] <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.tile_off[mid] <= t)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    b = lo;
+    load_seq(p);
+    const int r = static_cast<int>(t - p.tile_off[b]);
+    g = r / nt;
+    i = r - g * nt;
+  }
+  // Advance one tile (the caller never advances past its range's last tile).
+  __device__ __forceinline__ void next(const PParams& p) {
+    if (++i < nt) return;
+    i = 0;
+    if (++g < p.Hkv) return;
+    g = 0;
+    do {
+      ++b;
+    } while (b < p.B - 1 && p.tile_off[b + 1] == p.tile_off[b]);
+    load_seq(p);
+  }
+  __device__ __forceinline__ int segment(const PParams& p) const { return b * p.Hkv + g; }
+};
+
+template <int NP>
+struct PCfg {
+  static_assert(NP == 16 || NP == 32, "padded group");
+  static constexpr int kBoxBytes = TK * 128;          // 128 keys x 64 dims
+  static constexpr int kTileBytes = 2 * kBoxBytes;    // K or V tile (32 KB)
+  static constexpr int kStageBytes = 2 * kTileBytes;  // K tile, then V tile
+  static constexpr int kQBox = NP * 128;              // NP rows x 64 dims (or 64 keys)
+  static constexpr int kQBuf = 2 * kQBox;             // one Q (128 dims)
+  static constexpr int kQOff = kStages * kStageBytes;
+  static constexpr int kPBuf = 2 * kQBox;             // P^T: 2 boxes of 64 keys
+  static constexpr int kPOff = kQOff + 2 * kQBuf;
+  static constexpr int kRedOff = kPOff + 2 * kPBuf;   // [2][warps][NP] floats
+  // full[S], empty[S], s_ready[2], p_ready[2], x_bar[2], q_full[2], q_free[2], pv_done, drain
+  static constexpr int kBarOff = kRedOff + 2 * kSoftWarps * NP * 4;
+  static constexpr int kNumBars = 2 * kStages + 10 + 2;
+  static constexpr int kCtlOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kCtlOff + 64 + 1024;  // + runtime 1024-byte alignment
+  static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0 && kQBox % 1024 == 0, "swizzle atoms");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+template <int NP, typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_q, const PParams p) {
+  using C = PCfg<NP>;
+  using decode_tc::sw128_off;
+  using decode_tc::tmem_ld_np;
+  using decode_tc::tmem_st_np;
+  using decode_tc::to_bits;
+  using decode_tc::pick;
+  const int c = blockIdx.x;
+  const Range rg = cta_range(p, c, gridDim.x);
+  if (rg.lo >= rg.hi) return;  // no tiles for this CTA (uniform over the CTA)
+  const int n = static_cast<int>(rg.hi - rg.lo);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sQ = smem + C::kQOff;
+  uint8_t* sP = smem + C::kPOff;
+  float* red = reinterpret_cast<float*>(smem + C::kRedOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* full = bars;
+  uint64_t* empty = full + kStages;
+  uint64_t* s_ready = empty + kStages;
+  uint64_t* p_ready = s_ready + 2;
+  uint64_t* x_bar = p_ready + 2;
+  uint64_t* q_full = x_bar + 2;
+  uint64_t* q_free = q_full + 2;
+  uint64_t* pv_done = q_free + 2;
+  uint64_t* drain = pv_done + 1;
+  CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem + C::kCtlOff);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kCtlOff + 32);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 32);  // one cp.async arrival per producer lane
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_ready[i], 1);
+      mbar_init(&p_ready[i], 32 * kSoftWarps);
+      mbar_init(&x_bar[i], 32 * kSoftWarps);
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_free[i], 1);
+    }
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    ctl->abort = 0;
+    ctl->wait_ns = p.wait_ns;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+    if (lane == 0) tma_prefetch_desc(&tm_q);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tS0 = tmem;          // S^T buffers: columns [0, NP), [NP, 2 NP)
+  const uint32_t tO = tmem + 2 * NP;  // O^T: columns [2 NP, 3 NP)
+  const int G = p.G;
+
+  Cursor cur;
+  cur.seek(p, rg.lo);
+
+  if (warp >= kProdWarp0) {
+    // ------------------------------------------------------------ producers
+    // Producer pw fills stage pw with the CTA's tiles pw, pw + 3, ... Lane l
+    // copies 16-byte unit (l % 16) of rows 2i + l / 16: each instruction reads
+    // two whole 256-byte cache rows.
+    const int pw = warp - kProdWarp0;
+    bool ok = true;
+    const uint32_t kdst = smem_u32(smem + pw * C::kStageBytes);
+    const uint32_t vdst = kdst + C::kTileBytes;
+    const int u = lane & 15;
+    for (int a = 0; a < pw && a + 1 < n; ++a) cur.next(p);  // to tile pw (if in range)
+    for (int j = pw; ok && j < n; j += kStages) {
+      const int use = j / kStages;
+      if (use > 0 &&
+          !(ok = decode::warp_all_d(wait_bar(&empty[pw], (use - 1) & 1, ctl, kSiteEmpty))))
+        break;
+      const size_t head_base =
+          (static_cast<size_t>(cur.tok) * p.Hkv + static_cast<size_t>(cur.g) * cur.len) * D;
+      const T* kbase = reinterpret_cast<const T*>(p.kc) + head_base;
+      const T* vbase = reinterpret_cast<const T*>(p.vc) + head_base;
+      const int t0 = cur.k0 + cur.i * TK;
+#pragma unroll 4
+      for (int i = 0; i < TK / 2; ++i) {
+        const int r = 2 * i + (lane >> 4);
+        const int key = t0 + r;
+        const bool valid = key < cur.len;
+        const size_t row = static_cast<size_t>(valid ? key : t0);  // t0 < len: a real row
+        const uint32_t nb = valid ? 16u : 0u;                     // 0: zero-fill, no read
+        const uint32_t off = sw128_off(r, u, C::kBoxBytes);
+        cp_async16(kdst + off, kbase + row * D + u * 8, nb);
+        cp_async16(vdst + off, vbase + row * D + u * 8, nb);
+      }
+      cp_async_mbar_arrive_noinc(&full[pw]);
+      for (int a = 0; a < kStages && j + 1 + a < n; ++a) cur.next(p);
+    }
+    cp_async_wait_all();  // no copy may land after the CTA exits
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue and Q loads
+    constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+    constexpr uint32_t idesc_s = umma_idesc_f16(fmt, TK, NP, 0, 0);
+    constexpr uint32_t idesc_pv = umma_idesc_f16(fmt, D, NP, 1, 0);
+    const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+    const uint32_t d_hi = static_cast<uint32_t>(dq >> 32);
+    const uint32_t q_lo = static_cast<uint32_t>(dq);
+    const uint32_t k_lo = static_cast<uint32_t>(smem_desc_sw128(smem_u32(smem), 16, 1024));
+    const uint32_t v_lo = static_cast<uint32_t>(
+        smem_desc_sw128(smem_u32(smem + C::kTileBytes), C::kBoxBytes, 1024));
+    const uint32_t p_lo = static_cast<uint32_t>(smem_desc_sw128(smem_u32(sP), 16, 1024));
+    // Q of piece k goes to buffer k % 2 (its G rows; rows G..NP-1 are zero-filled
+    // by the copy as out of bounds). The first piece's Q is loaded here.
+    int nq[2] = {0, 0};  // Q loads issued per buffer
+    auto load_q = [&](int buf, int seg) {
+      ++nq[buf];
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&q_full[buf], 2 * C::kQBox);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_3d(sQ + buf * C::kQBuf + bx * C::kQBox, &tm_q, &q_full[buf], bx * 64, 0, seg);
+      }
+      __syncwarp();
+    };
+    load_q(0, cur.segment(p));
+    bool ok = true;
+    int k = -1;                // current piece
+    bool prev_first = false;   // tile j - 1 started its piece
+    uint32_t qb = 0;
+    for (int j = 0; ok && j <= n; ++j) {
+      if (j < n) {
+        const bool first = (j == 0) || (cur.i == 0);
+        const bool last = (j == n - 1) || (cur.i == cur.nt - 1);
+        if (first) {
+          ++k;
+          qb = k & 1;
+          if (!(ok = decode::warp_all_d(wait_bar(&q_full[qb], (k >> 1) & 1, ctl, kSiteQ)))) break;
+          tc_fence_after();
+        }
+        // S^T(j) = K_j Q^T into buffer j % 2 (its previous scores, of tile
+        // j - 2, were read before p_ready(j - 2), waited for last iteration).
+        const int st = j % kStages;
+        if (!(ok = decode::warp_all_d(wait_bar(&full[st], (j / kStages) & 1, ctl, kSiteFull))))
+          break;
+        fence_proxy_async_smem();  // the cp.async data is read by the tensor core
+        tc_fence_after();
+        const uint32_t kd = k_lo + ((st * C::kStageBytes) >> 4);
+        const uint32_t qd = q_lo + ((qb * C::kQBuf) >> 4);
+        const uint32_t tS = tS0 + (j & 1) * NP;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+          const uint32_t qo = ((kk >> 2) * C::kQBox + (kk & 3) * 32) >> 4;
+          if (kk == 0)
+            umma_ss_w<0>(tS, desc_words(kd + ko, d_hi), desc_words(qd + qo, d_hi), idesc_s);
+          else
+            umma_ss_w<1>(tS, desc_words(kd + ko, d_hi), desc_words(qd + qo, d_hi), idesc_s);
+        }
+        umma_commit_w(&s_ready[j & 1]);
+        if (last) umma_commit_w(&q_free[qb]);  // Q buffer free once this product is done
+        if (first && j + (cur.nt - cur.i) < n) {
+          // Load the next piece's Q into the other buffer, which piece k - 1
+          // used: wait until its last score product has read it.
+          Cursor nx = cur;  // first tile of the next piece, tile j + nt - i (< n)
+          for (int a = cur.i; a < cur.nt; ++a) nx.next(p);
+          if (k >= 1 && !(ok = decode::warp_all_d(
+                              wait_bar(&q_free[qb ^ 1], ((k - 1) >> 1) & 1, ctl, kSiteQFree))))
+            break;
+          load_q(qb ^ 1, nx.segment(p));
+        }
+      }
+      if (j >= 1) {
+        // O^T (+)= V_{j-1}^T P^T(j-1); then stage (j-1) % 3 is free again.
+        const int jp = j - 1;
+        const int st = jp % kStages;
+        if (!(ok = decode::warp_all_d(wait_bar(&p_ready[jp & 1], (jp >> 1) & 1, ctl, kSiteP))))
+          break;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t vd = v_lo + ((st * C::kStageBytes) >> 4);
+        const uint32_t pd = p_lo + (((jp & 1) * C::kPBuf) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < TK / 16; ++kk) {
+          const uint32_t vo = kk * 128;  // 16 keys = 16 rows of 128 bytes
+          const uint32_t po = ((kk >> 2) * C::kQBox + (kk & 3) * 32) >> 4;
+          if (prev_first && kk == 0)
+            umma_ss_w<0>(tO, desc_words(vd + vo, d_hi), desc_words(pd + po, d_hi), idesc_pv);
+          else
+            umma_ss_w<1>(tO, desc_words(vd + vo, d_hi), desc_words(pd + po, d_hi), idesc_pv);
+        }
+        umma_commit_w(&empty[st]);
+        umma_commit_w(pv_done);
+      }
+      if (j < n) {
+        prev_first = (j == 0) || (cur.i == 0);
+        if (j + 1 < n) cur.next(p);
+      }
+    }
+    // Every MMA and every Q copy must be complete before the CTA exits (a
+    // copy issued for a piece is waited for when the piece starts, except on
+    // the abort path).
+    umma_commit_w(drain);
+    drain_bar(drain, 0, ctl, kSiteDrain);
+    for (int buf = 0; buf < 2; ++buf)
+      if (nq[buf] > 0) drain_bar(&q_full[buf], (nq[buf] - 1) & 1, ctl, kSiteDrain);
+  } else {
+    // ------------------------------------------------------------ softmax and epilogue
+    const int krow = warp * 32 + lane;  // this thread's key in a tile (tensor-memory lane)
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    float m[NP], l[NP];
+    bool ok = true;
+    uint32_t xc = 0;        // uses of the x_bar / red exchange so far
+    bool piece_whole = false;
+    for (int j = 0; j < n; ++j) {
+      const bool first = (j == 0) || (cur.i == 0);
+      const bool last = (j == n - 1) || (cur.i == cur.nt - 1);
+      if (first) {
+        piece_whole = (cur.i == 0);
+#pragma unroll
+        for (int h = 0; h < NP; ++h) {
+          m[h] = -INFINITY;
+          l[h] = 0.f;
+        }
+      }
+      if (last) piece_whole = piece_whole && (cur.i == cur.nt - 1);
+      if (!(ok = decode::warp_all_d(wait_bar(&s_ready[j & 1], (j >> 1) & 1, ctl, kSiteS)))) break;
+      tc_fence_after();
+      uint32_t r[NP];
+      tmem_ld_np<NP>(tS0 + lane_off + (j & 1) * NP, r);
+      const bool valid = cur.k0 + cur.i * TK + krow < cur.len;
+      float s[NP], wm[NP];
+#pragma unroll
+      for (int h = 0; h < NP; ++h) {
+        s[h] = (valid && h < G) ? __uint_as_float(r[h]) * sl2 : -INFINITY;
+        wm[h] = s[h];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int h = 0; h < NP; ++h) wm[h] = fmaxf(wm[h], __shfl_xor_sync(0xffffffffu, wm[h], o));
+      float* rb = red + (xc & 1) * (kSoftWarps * NP);
+      if (lane < NP) rb[warp * NP + lane] = pick<NP>(wm, lane);
+      mbar_arrive(&x_bar[xc & 1]);
+      if (!(ok = decode::warp_all_d(wait_bar(&x_bar[xc & 1], (xc >> 1) & 1, ctl, kSiteX)))) break;
+      ++xc;
+      float alpha[NP];
+      bool rescale = false;
+#pragma unroll
+      for (int h = 0; h < NP; ++h) {
+        const float tm = fmaxf(fmaxf(rb[h], rb[NP + h]), fmaxf(rb[2 * NP + h], rb[3 * NP + h]));
+        alpha[h] = 1.f;
+        if (tm > m[h] + kRescaleThreshold) {
+          alpha[h] = ex2_approx(m[h] - tm);  // m = -inf gives 0
+          m[h] = tm;
+          l[h] *= alpha[h];
+          rescale = true;
+        }
+      }
+      if (rescale && !first) {
+        // O^T was last written by PV(j-1) of this piece; wait for it, then
+        // scale this warp's 32 dims by the heads' alpha.
+        if (!(ok = decode::warp_all_d(wait_bar(pv_done, (j - 1) & 1, ctl, kSitePv)))) break;
+        tc_fence_after();
+        uint32_t o[NP];
+        tmem_ld_np<NP>(tO + lane_off, o);
+#pragma unroll
+        for (int h = 0; h < NP; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+        tmem_st_np<NP>(tO + lane_off, o);
+        tmem_wait_st();
+      }
+      // P^T(j): row h, key krow, in buffer j % 2 (read by PV(j - 2), which
+      // completed before S(j) was signalled).
+      uint8_t* pb = sP + (j & 1) * C::kPBuf + (krow >> 6) * C::kQBox;
+      const int kc = krow & 63;
+#pragma unroll
+      for (int h = 0; h < NP; ++h) {
+        float pv = 0.f;
+        if (h < G) {
+          pv = ex2_approx(s[h] - (m[h] == -INFINITY ? 0.f : m[h]));
+          l[h] += pv;
+        }
+        *reinterpret_cast<uint16_t*>(pb + h * 128 + ((((kc >> 3) ^ (h & 7))) << 4) +
+                                     ((kc & 7) << 1)) = to_bits<T>(pv);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_ready[j & 1]);
+
+      if (last) {
+        // ---- end of a piece: row sums over the tile's 128 key slots, then O.
+        float lt[NP];
+#pragma unroll
+        for (int h = 0; h < NP; ++h) lt[h] = l[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int h = 0; h < NP; ++h) lt[h] += __shfl_xor_sync(0xffffffffu, lt[h], o);
+        float* rl = red + (xc & 1) * (kSoftWarps * NP);
+        if (lane < NP) rl[warp * NP + lane] = pick<NP>(lt, lane);
+        mbar_arrive(&x_bar[xc & 1]);
+        if (!(ok = decode::warp_all_d(wait_bar(&x_bar[xc & 1], (xc >> 1) & 1, ctl, kSiteX)))) break;
+        ++xc;
+        if (!(ok = decode::warp_all_d(wait_bar(pv_done, j & 1, ctl, kSitePv)))) break;
+        tc_fence_after();
+        uint32_t o[NP];
+        tmem_ld_np<NP>(tO + lane_off, o);
+        const int dim = krow;  // O^T lane = output dimension
+        const int seg = cur.segment(p);
+        const size_t row0 = static_cast<size_t>(cur.b) * p.Hq + static_cast<size_t>(cur.g) * G;
+#pragma unroll
+        for (int h = 0; h < NP; ++h) {
+          if (h < G) {
+            const float tot = rl[h] + rl[NP + h] + rl[2 * NP + h] + rl[3 * NP + h];
+            const float ov = tot > 0.f ? __uint_as_float(o[h]) / tot : 0.f;
+            const float l2 = tot > 0.f ? m[h] + lg2_approx(tot) : -INFINITY;
+            if (piece_whole) {
+              // The whole segment lay in this CTA: this is the result.
+              reinterpret_cast<uint16_t*>(p.o)[(row0 + h) * D + dim] = to_bits<T>(ov);
+              if (dim == h && p.lse != nullptr) p.lse[row0 + h] = l2 * 0.69314718055994531f;
+            } else {
+              const size_t slot = static_cast<size_t>(seg) + c;
+              p.part_o[(slot * G + h) * D + dim] = ov;
+              if (dim == h) p.part_lse[slot * G + h] = l2;
+            }
+          }
+        }
+        // O^T is overwritten by the next piece's first product only after
+        // that piece's first p_ready, which follows this read.
+        tc_fence_before();
+      }
+      if (j + 1 < n) cur.next(p);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ gather
+// One warp per (sequence b, query head h): a segment cut between CTAs (in the
+// equal-tile-range mode) has one partial per CTA, in slots segment + cta;
+// merge them by their log-sum-exp. An empty sequence gets O = 0, LSE = -inf.
+// Segments that lay in one CTA were written by it and are skipped.
+template <typename T>
+__global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p, int nc) {
+  const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(p.B) * p.Hq) return;
+  const int b = static_cast<int>(row / p.Hq);
+  const int h = static_cast<int>(row - static_cast<long long>(b) * p.Hq);
+  const int g = h / p.G;
+  const int hh = h - g * p.G;
+  const int nt = (p.tile_off[b + 1] - p.tile_off[b]) / p.Hkv;
+  T* dst = reinterpret_cast<T*>(p.o) + row * D + lane * 4;
+  if (nt == 0) {
+    uint2 z;
+    z.x = decode::pack2<T>(0.f, 0.f);
+    z.y = z.x;
+    *reinterpret_cast<uint2*>(dst) = z;
+    if (lane == 0 && p.lse != nullptr) p.lse[row] = -INFINITY;
+    return;
+  }
+  if (p.seg_aligned) return;
+  const long long T_all = p.tile_off[p.B];
+  const long long a = p.tile_off[b] + static_cast<long long>(g) * nt;
+  const int c0 = cta_of(a, T_all, nc);
+  const int c1 = cta_of(a + nt - 1, T_all, nc);
+  if (c0 == c1) return;
+  const long long seg = static_cast<long long>(b) * p.Hkv + g;
+  // CTAs between c0 and c1 with an empty tile range (fewer tiles than CTAs)
+  // wrote nothing: their slots are skipped.
+  auto has_tiles = [&](int cc) { return cc * T_all / nc < (cc + 1) * T_all / nc; };
+  float mx = -INFINITY;
+  for (int cc = c0; cc <= c1; ++cc)
+    if (has_tiles(cc)) mx = fmaxf(mx, p.part_lse[(seg + cc) * p.G + hh]);
+  float tot = 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (mx != -INFINITY) {
+    for (int cc = c0; cc <= c1; ++cc) {
+      if (!has_tiles(cc)) continue;
+      const long long slot = (seg + cc) * p.G + hh;
+      const float wt = ex2_approx(p.part_lse[slot] - mx);
+      tot += wt;
+      const float4 x = *reinterpret_cast<const float4*>(p.part_o + slot * D + lane * 4);
+      acc[0] = fmaf(wt, x.x, acc[0]);
+      acc[1] = fmaf(wt, x.y, acc[1]);
+      acc[2] = fmaf(wt, x.z, acc[2]);
+      acc[3] = fmaf(wt, x.w, acc[3]);
+    }
+  }
+  const float inv = tot > 0.f ? 1.f / tot : 0.f;
+  uint2 pk;
+  pk.x = decode::pack2<T>(acc[0] * inv, acc[1] * inv);
+  pk.y = decode::pack2<T>(acc[2] * inv, acc[3] * inv);
+  *reinterpret_cast<uint2*>(dst) = pk;
+  if (lane == 0 && p.lse != nullptr)
+    p.lse[row] = tot > 0.f ? (mx + lg2_approx(tot)) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace decode_ps
+}  // namespace eta

@@ -164,3 +164,36 @@ def test_decode_tensor_core_single_split_writes_output(lib):
     compare(o, lse, o_ref, lse_ref, F16, "single split")
     o2, none = run(lib, *args, want_lse=False)
     assert none is None and torch.equal(o, o2)
+
+
+# The persistent pass divides all (sequence, KV head) tiles of 128 keys into
+# equal contiguous ranges, one per CTA; segments cut between CTAs are merged by
+# the gather kernel. These cases stress the cuts.
+PS_CASES = [
+    # B, Hq, Hkv, lengths, dtype
+    (1, 8, 1, [1000], BF16),                  # 8 tiles over every CTA: most CTAs own none
+    (3, 32, 2, [70000, 5, 300], BF16),        # one long segment cut over many CTAs
+    (300, 16, 2, "short", F16),               # many short sequences, empties between
+    (64, 32, 1, "ragged", BF16),              # MQA at the workload's scale
+    (64, 128, 8, "ragged", BF16),             # group 16 at the workload's scale
+]
+
+
+@pytest.mark.parametrize("case", PS_CASES, ids=lambda c: f"B{c[0]}h{c[1]}kv{c[2]}")
+def test_decode_persistent_cuts(lib, case):
+    B, Hq, Hkv, lens, dt = case
+    if lens == "short":
+        sl = workloads.decode_seqlens(B, 0, 200, 2500)
+        sl[::7] = 0
+    elif lens == "ragged":
+        sl = workloads.decode_seqlens(B, 1024, 8192, 2501)
+    else:
+        sl = torch.tensor(lens, dtype=torch.int32)
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, 128, sl, dt,
+                                            seed=2600 + PS_CASES.index(case))
+    scale = 128 ** -0.5
+    o, lse = run(lib, q.to(DEV), kc.to(DEV), vc.to(DEV), sl.to(DEV), Hkv, scale)
+    o2, lse2 = run(lib, q.to(DEV), kc.to(DEV), vc.to(DEV), sl.to(DEV), Hkv, scale)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)  # fixed assignment: bitwise repeatable
+    o_ref, lse_ref = oracle.decode_ref(q, kc, vc, sl, scale, Hkv)
+    compare(o, lse, o_ref, lse_ref, dt, f"persistent {case[:3]}")

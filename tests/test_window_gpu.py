@@ -58,6 +58,7 @@ DECODE = [
     (3, 32, 8, 128, [5000, 100, 2049], 1000, BF16),
     (2, 16, 2, 64, [129, 4096], 129, F16),
     (2, 8, 1, 128, [777, 20], 1, BF16),
+    (5, 64, 4, 128, [9000, 0, 130, 4000, 257], 1100, BF16),  # group 16, persistent pass
 ]
 
 

@@ -73,27 +73,29 @@ def _oracle_sample(q, kc, vc, sl, Hkv, o, lse, seqs, what):
         compare(o[b:b + 1], lse[b:b + 1], o_ref, l_ref, torch.bfloat16, f"{what} seq {b}")
 
 
-def test_noalloc_fewer_splits_than_usual(lib):
-    # One split of B=128, Hq=32, d=128 needs 528,384 floats: 3 fit in the
-    # scratch, while attn_decode uses 4 splits here on a 148-SM B200.
-    B, Hq, Hkv, d = 128, 32, 8, 128
-    per_split = B * Hq * (d + 1)
-    fit = 2_097_152 // per_split
-    want = lib.attn_decode_num_splits(B, Hq, Hkv, d)
-    assert fit == 3 and want > fit, (fit, want)
+def test_noalloc_persistent_partials_fill_most_of_the_scratch(lib):
+    # The persistent pass (d = 128, 2..32 query heads per KV head) keeps its
+    # plan and the partials of segments cut between CTAs in the scratch:
+    # (B * Hkv + CTAs - 1) slots of G rows of d + 1 floats, one CTA per SM.
+    # B=44, Hq=256, Hkv=8 (group 32) needs about 7.9 MiB of the 8 MiB.
+    B, Hq, Hkv, d = 44, 256, 8, 128
+    G = Hq // Hkv
+    slots = B * Hkv + torch.cuda.get_device_properties(0).multi_processor_count - 1
+    assert slots * G * (d + 1) < 2_097_152 < (slots + 40) * G * (d + 1)
     sl = workloads.decode_seqlens(B, 1, 3000, 47)
     q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, d, sl, torch.bfloat16, seed=47,
                                             device=DEV)
     _call_pair(lib, q, kc, vc, sl, Hkv)
     o, lse = lib.attn_decode_noalloc(q, kc, vc, sl, Hkv=Hkv)
     torch.cuda.synchronize()
-    _oracle_sample(q, kc, vc, sl, Hkv, o, lse, range(0, B, 9), "noalloc 3 of 4 splits")
+    _oracle_sample(q, kc, vc, sl, Hkv, o, lse, range(0, B, 5), "noalloc persistent group 32")
 
 
 def test_noalloc_tensor_core_single_split_beyond_scratch(lib):
-    # Groups of 8..32 heads at d = 128 with one split per sequence need no
-    # scratch: even sizes where one split would not fit the array run (this one
-    # needs 4096 * 32 * 129 floats per split, about 8 times the array).
+    # Groups of 2..32 heads at d = 128 run on the persistent pass, whose
+    # partials would need (4096 * 4 + 147) * 8 * 129 floats here, about 8 times
+    # the array: every CTA then takes whole segments and writes its results
+    # directly, with only the per-sequence plan in the scratch.
     B, Hq, Hkv, d = 4096, 32, 4, 128
     assert B * Hq * (d + 1) > 2_097_152
     assert lib.attn_decode_num_splits(B, Hq, Hkv, d) == 1
@@ -107,9 +109,9 @@ def test_noalloc_tensor_core_single_split_beyond_scratch(lib):
 
 
 def test_noalloc_refuses_sizes_beyond_its_scratch(lib):
-    # B * Hq * (d + 1) floats per split on the CUDA-core pass (4 query heads
+    # B * Hq * (d + 1) floats per split on the CUDA-core pass (one query head
     # per KV head); 16384 * 8 * 129 is above 2,097,152.
-    B, Hq, Hkv, d = 16384, 8, 2, 128
+    B, Hq, Hkv, d = 16384, 8, 8, 128
     q = torch.zeros(B, Hq, d, device=DEV, dtype=torch.bfloat16)
     kc = torch.zeros(64, device=DEV, dtype=torch.bfloat16)
     sl = torch.zeros(B, device=DEV, dtype=torch.int32)
