@@ -447,10 +447,10 @@ int launch_decode_tc(const decode::DParams& p, cudaStream_t st) {
 
 // Plan, persistent stream and gather of the d = 128 decode; `ws` holds the
 // layout `L`. seg_aligned: whole segments per CTA (L has no partials).
-template <int NP, typename T>
+template <int NP, int GP, typename T>
 int launch_decode_ps(const CUtensorMap& tq, decode_ps::PParams p, const PsLayout& L, char* ws,
                      int nc, cudaStream_t st) {
-  auto kern = decode_ps::attn_decode_persistent_kernel<NP, T>;
+  auto kern = decode_ps::attn_decode_persistent_kernel<NP, GP, T>;
   constexpr int smem = decode_ps::PCfg<NP>::kSmemBytes;
   static PerDeviceOnce attr;
   const cudaError_t attr_err = attr.run([&]() {
@@ -467,12 +467,27 @@ int launch_decode_ps(const CUtensorMap& tq, decode_ps::PParams p, const PsLayout
       p.seqlens, tok_off, tile_off, p.B, p.Hkv, p.window);
   int rc = launch_status();
   if (rc != ATTN_OK) return rc;
-  kern<<<nc, decode_ps::kThreads, smem, st>>>(tq, p);
-  rc = launch_status();
-  if (rc != ATTN_OK) return rc;
+  // The stream and gather kernels are launched as programmatic dependents:
+  // each may start before the previous kernel ends and waits on the device
+  // (griddepcontrol.wait) for its results, so launch gaps overlap work.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nc));
+  cfg.blockDim = dim3(decode_ps::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, p);
+  if (e != cudaSuccess) return cuda_fail(e);
   const long long rows = static_cast<long long>(p.B) * p.Hq;
-  decode_ps::attn_decode_gather_kernel<T>
-      <<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(p, nc);
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&cfg, decode_ps::attn_decode_gather_kernel<T>, p, nc);
+  if (e != cudaSuccess) return cuda_fail(e);
   return launch_status();
 }
 
@@ -506,8 +521,10 @@ int decode_ps_run(const void* q, const void* kc, const void* vc, const int32_t* 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
   const PsLayout L = ps_layout(B, Hkv, G, nc, !seg_aligned);
-  return NP == 16 ? launch_decode_ps<16, T>(tq, p, L, ws, nc, st)
-                  : launch_decode_ps<32, T>(tq, p, L, ws, nc, st);
+  if (G <= 4) return launch_decode_ps<16, 4, T>(tq, p, L, ws, nc, st);
+  if (G <= 8) return launch_decode_ps<16, 8, T>(tq, p, L, ws, nc, st);
+  if (G <= 16) return launch_decode_ps<16, 16, T>(tq, p, L, ws, nc, st);
+  return launch_decode_ps<32, 32, T>(tq, p, L, ws, nc, st);
 }
 
 template <int D, typename T>

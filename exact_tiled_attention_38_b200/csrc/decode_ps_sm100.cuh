@@ -101,6 +101,15 @@ struct PParams {
   uint64_t wait_ns;
 };
 
+// Programmatic dependent launch: a grid launched with programmatic stream
+// serialisation may start before the previous kernel on the stream ends;
+// griddepcontrol.wait blocks until that kernel has completed and its memory
+// writes are visible, and launch_dependents lets the next such grid start.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Keys of sequence b read: [first_key, len).
 __device__ __forceinline__ int first_key(int len, int window) {
   return (window > 0 && len > window) ? len - window : 0;
@@ -116,6 +125,7 @@ __global__ void __launch_bounds__(kPlanThreads) attn_decode_plan_kernel(const in
                                                                       int B, int Hkv, int window) {
   __shared__ long long s_tok[kPlanThreads / 32];
   __shared__ long long s_til[kPlanThreads / 32];
+  griddep_launch_dependents();  // the stream kernel may start its set-up now
   const int per = (B + kPlanThreads - 1) / kPlanThreads;  // consecutive sequences per thread
   const int b0 = threadIdx.x * per;
   const int b1 = min(B, b0 + per);
@@ -264,19 +274,73 @@ struct PCfg {
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
-template <int NP, typename T>
+struct MaxOp {
+  __device__ __forceinline__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+struct AddOp {
+  __device__ __forceinline__ float operator()(float a, float b) const { return a + b; }
+};
+
+// Combine v[0..GP) over the 32 lanes of the warp; lane l returns the result
+// for entry l % GP. Butterfly steps with offsets 16 .. GP combine whole
+// arrays; then each step with offset M < GP hands over half of the remaining
+// entries (a reduce-scatter): (GP - 1) + GP * log2(32 / GP) shuffles in all,
+// against 5 * GP for a full butterfly per entry.
+template <int GP, typename Op>
+__device__ __forceinline__ float reduce_scatter(float (&v)[GP], int lane, Op op) {
+#pragma unroll
+  for (int M = 16; M >= GP; M >>= 1)
+#pragma unroll
+    for (int j = 0; j < GP; ++j) v[j] = op(v[j], __shfl_xor_sync(0xffffffffu, v[j], M));
+#pragma unroll
+  for (int M = GP / 2; M >= 1; M >>= 1) {
+    const bool up = (lane & M) != 0;
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      const float send = up ? v[j] : v[j + M];
+      const float keep = up ? v[j + M] : v[j];
+      v[j] = op(keep, __shfl_xor_sync(0xffffffffu, send, M));
+    }
+  }
+  return v[0];
+}
+
+// out[h] = op over the four softmax warps of red[w * NP + h], h < GP, read as
+// 16-byte vectors (every thread reads the same words: broadcasts).
+template <int GP, int NP, typename Op>
+__device__ __forceinline__ void gather4(const float* red, float (&out)[GP], Op op) {
+  const float4* r4 = reinterpret_cast<const float4*>(red);
+#pragma unroll
+  for (int q = 0; q < GP / 4; ++q) {
+    float4 a = r4[q];
+#pragma unroll
+    for (int w = 1; w < kSoftWarps; ++w) {
+      const float4 b = r4[w * (NP / 4) + q];
+      a.x = op(a.x, b.x);
+      a.y = op(a.y, b.y);
+      a.z = op(a.z, b.z);
+      a.w = op(a.w, b.w);
+    }
+    out[4 * q] = a.x;
+    out[4 * q + 1] = a.y;
+    out[4 * q + 2] = a.z;
+    out[4 * q + 3] = a.w;
+  }
+}
+
+// NP: MMA width (the group padded to 16 or 32); GP <= NP: the heads the
+// softmax processes (the group padded to 4, 8, 16 or 32).
+template <int NP, int GP, typename T>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_q, const PParams p) {
+  static_assert(GP == 4 || GP == 8 || GP == 16 || GP == 32, "softmax group");
+  static_assert(GP <= NP && (GP > 16) == (NP == 32), "widths");
   using C = PCfg<NP>;
   using decode_tc::sw128_off;
   using decode_tc::tmem_ld_np;
   using decode_tc::tmem_st_np;
   using decode_tc::to_bits;
-  using decode_tc::pick;
   const int c = blockIdx.x;
-  const Range rg = cta_range(p, c, gridDim.x);
-  if (rg.lo >= rg.hi) return;  // no tiles for this CTA (uniform over the CTA)
-  const int n = static_cast<int>(rg.hi - rg.lo);
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -331,10 +395,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tO = tmem + 2 * NP;  // O^T: columns [2 NP, 3 NP)
   const int G = p.G;
 
+  // The plan is written by the kernel launched just before this one, which
+  // lets this grid start early (programmatic dependent launch): the set-up
+  // above overlaps it, and this wait returns once its writes are visible.
+  // The gather grid after this one may then start and wait in the same way.
+  griddep_wait();
+  griddep_launch_dependents();
+  const Range rg = cta_range(p, c, gridDim.x);
+  const int n = rg.hi > rg.lo ? static_cast<int>(rg.hi - rg.lo) : 0;  // tiles of this CTA
   Cursor cur;
-  cur.seek(p, rg.lo);
+  if (n > 0) cur.seek(p, rg.lo);
 
-  if (warp >= kProdWarp0) {
+  if (n == 0) {
+    // no tiles for this CTA (uniform over the CTA)
+  } else if (warp >= kProdWarp0) {
     // ------------------------------------------------------------ producers
     // Producer pw fills stage pw with the CTA's tiles pw, pw + 3, ... Lane l
     // copies 16-byte unit (l % 16) of rows 2i + l / 16: each instruction reads
@@ -477,10 +551,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (nq[buf] > 0) drain_bar(&q_full[buf], (nq[buf] - 1) & 1, ctl, kSiteDrain);
   } else {
     // ------------------------------------------------------------ softmax and epilogue
+    // Each thread holds the GP (>= G) head scores of its key. The padded rows
+    // GP..NP-1 of both P^T buffers are zeroed once here and never written
+    // again, so the products' padded columns stay zero.
     const int krow = warp * 32 + lane;  // this thread's key in a tile (tensor-memory lane)
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float sl2 = p.scale_log2;
-    float m[NP], l[NP];
+    if constexpr (GP < NP) {
+      for (int i = threadIdx.x; i < 2 * 2 * (NP - GP) * 8; i += 32 * kSoftWarps) {
+        const int chunk = i & 7, row = GP + ((i >> 3) % (NP - GP)), box = i / (8 * (NP - GP));
+        *reinterpret_cast<uint4*>(sP + box * C::kQBox + row * 128 + chunk * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+    }
+    float m[GP], l[GP];
     bool ok = true;
     uint32_t xc = 0;        // uses of the x_bar / red exchange so far
     bool piece_whole = false;
@@ -490,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (first) {
         piece_whole = (cur.i == 0);
 #pragma unroll
-        for (int h = 0; h < NP; ++h) {
+        for (int h = 0; h < GP; ++h) {
           m[h] = -INFINITY;
           l[h] = 0.f;
         }
@@ -501,30 +586,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t r[NP];
       tmem_ld_np<NP>(tS0 + lane_off + (j & 1) * NP, r);
       const bool valid = cur.k0 + cur.i * TK + krow < cur.len;
-      float s[NP], wm[NP];
+      float s[GP], wm[GP];
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
+      for (int h = 0; h < GP; ++h) {
         s[h] = (valid && h < G) ? __uint_as_float(r[h]) * sl2 : -INFINITY;
         wm[h] = s[h];
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int h = 0; h < NP; ++h) wm[h] = fmaxf(wm[h], __shfl_xor_sync(0xffffffffu, wm[h], o));
+      // tile max per head: this warp's 32 keys by a reduce-scatter (lane l ends
+      // with head l % GP), then the four warps through shared memory
+      const float wmax = reduce_scatter<GP>(wm, lane, MaxOp());
       float* rb = red + (xc & 1) * (kSoftWarps * NP);
-      if (lane < NP) rb[warp * NP + lane] = pick<NP>(wm, lane);
+      if (lane < GP) rb[warp * NP + lane] = wmax;
       mbar_arrive(&x_bar[xc & 1]);
       if (!(ok = decode::warp_all_d(wait_bar(&x_bar[xc & 1], (xc >> 1) & 1, ctl, kSiteX)))) break;
       ++xc;
-      float alpha[NP];
+      float tm[GP];
+      gather4<GP, NP>(rb, tm, MaxOp());
+      float alpha[GP];
       bool rescale = false;
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
-        const float tm = fmaxf(fmaxf(rb[h], rb[NP + h]), fmaxf(rb[2 * NP + h], rb[3 * NP + h]));
+      for (int h = 0; h < GP; ++h) {
         alpha[h] = 1.f;
-        if (tm > m[h] + kRescaleThreshold) {
-          alpha[h] = ex2_approx(m[h] - tm);  // m = -inf gives 0
-          m[h] = tm;
+        if (tm[h] > m[h] + kRescaleThreshold) {
+          alpha[h] = ex2_approx(m[h] - tm[h]);  // m = -inf gives 0
+          m[h] = tm[h];
           l[h] *= alpha[h];
           rescale = true;
         }
@@ -537,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t o[NP];
         tmem_ld_np<NP>(tO + lane_off, o);
 #pragma unroll
-        for (int h = 0; h < NP; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+        for (int h = 0; h < GP; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
         tmem_st_np<NP>(tO + lane_off, o);
         tmem_wait_st();
       }
@@ -546,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* pb = sP + (j & 1) * C::kPBuf + (krow >> 6) * C::kQBox;
       const int kc = krow & 63;
 #pragma unroll
-      for (int h = 0; h < NP; ++h) {
+      for (int h = 0; h < GP; ++h) {
         float pv = 0.f;
         if (h < G) {
           pv = ex2_approx(s[h] - (m[h] == -INFINITY ? 0.f : m[h]));
@@ -561,18 +646,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (last) {
         // ---- end of a piece: row sums over the tile's 128 key slots, then O.
-        float lt[NP];
+        float lt[GP];
 #pragma unroll
-        for (int h = 0; h < NP; ++h) lt[h] = l[h];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-          for (int h = 0; h < NP; ++h) lt[h] += __shfl_xor_sync(0xffffffffu, lt[h], o);
+        for (int h = 0; h < GP; ++h) lt[h] = l[h];
+        const float wsum = reduce_scatter<GP>(lt, lane, AddOp());
         float* rl = red + (xc & 1) * (kSoftWarps * NP);
-        if (lane < NP) rl[warp * NP + lane] = pick<NP>(lt, lane);
+        if (lane < GP) rl[warp * NP + lane] = wsum;
         mbar_arrive(&x_bar[xc & 1]);
         if (!(ok = decode::warp_all_d(wait_bar(&x_bar[xc & 1], (xc >> 1) & 1, ctl, kSiteX)))) break;
         ++xc;
+        float tot[GP];
+        gather4<GP, NP>(rl, tot, AddOp());
         if (!(ok = decode::warp_all_d(wait_bar(pv_done, j & 1, ctl, kSitePv)))) break;
         tc_fence_after();
         uint32_t o[NP];
@@ -581,11 +665,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int seg = cur.segment(p);
         const size_t row0 = static_cast<size_t>(cur.b) * p.Hq + static_cast<size_t>(cur.g) * G;
 #pragma unroll
-        for (int h = 0; h < NP; ++h) {
+        for (int h = 0; h < GP; ++h) {
           if (h < G) {
-            const float tot = rl[h] + rl[NP + h] + rl[2 * NP + h] + rl[3 * NP + h];
-            const float ov = tot > 0.f ? __uint_as_float(o[h]) / tot : 0.f;
-            const float l2 = tot > 0.f ? m[h] + lg2_approx(tot) : -INFINITY;
+            const float ov = tot[h] > 0.f ? __uint_as_float(o[h]) / tot[h] : 0.f;
+            const float l2 = tot[h] > 0.f ? m[h] + lg2_approx(tot[h]) : -INFINITY;
             if (piece_whole) {
               // The whole segment lay in this CTA: this is the result.
               reinterpret_cast<uint16_t*>(p.o)[(row0 + h) * D + dim] = to_bits<T>(ov);
@@ -621,6 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Segments that lay in one CTA were written by it and are skipped.
 template <typename T>
 __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p, int nc) {
+  griddep_wait();  // the stream kernel's partials and outputs are visible after this
   const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= static_cast<long long>(p.B) * p.Hq) return;
