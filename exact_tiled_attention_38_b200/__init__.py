@@ -45,6 +45,10 @@ SIGNATURES = {
     "attn_last_cuda_error": (_I, []),
     "attn_merge": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _P]),
     "attn_merge_f16": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _P]),
+    "attn_fwd_partial": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_fwd_partial_f16": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_merge_partial": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _P]),
+    "attn_merge_partial_f16": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _I, _P]),
 }
 
 _lib = None
@@ -113,9 +117,11 @@ def _on_device(*tensors):
     return torch.cuda.device(next(iter(devs)))
 
 
-def _fwd(fname, dtype, q, k, v, o, lse, scale, causal, stream, want_lse, window=None):
+def _fwd(fname, dtype, q, k, v, o, lse, scale, causal, stream, want_lse, window=None,
+         out_dtype=None):
     import torch
 
+    out_dtype = out_dtype or dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
         if t.dtype != dtype or t.dim() != 4:
@@ -127,10 +133,10 @@ def _fwd(fname, dtype, q, k, v, o, lse, scale, causal, stream, want_lse, window=
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, device=q.device, dtype=out_dtype)
     _dev(o, "o")
-    if o.dtype != dtype or tuple(o.shape) != tuple(q.shape):
-        raise ValueError("o must match q")
+    if o.dtype != out_dtype or tuple(o.shape) != tuple(q.shape):
+        raise ValueError(f"o must be a {out_dtype} tensor of q's shape")
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32)
     if lse is not None:
@@ -162,6 +168,21 @@ def attn_fwd_f16(q, k, v, o=None, lse=None, scale: Optional[float] = None,
 
     return _fwd("attn_fwd_f16", torch.float16, q, k, v, o, lse, scale, causal, stream,
                 want_lse)
+
+
+def attn_fwd_partial(q, k, v, o=None, lse=None, scale: Optional[float] = None,
+                     causal: bool = False, stream=None, want_lse: bool = True) -> Tuple:
+    """Prefill attention with O kept in float32 (unrounded), for results that
+    are merged further (``attn_merge`` with a float32 ``o_part``). q, k, v bf16
+    or fp16; returns (o float32 [B,Hq,Nq,d], lse)."""
+    import torch
+
+    if q.dtype == torch.float16:
+        name, dt = "attn_fwd_partial_f16", torch.float16
+    else:
+        name, dt = "attn_fwd_partial", torch.bfloat16
+    return _fwd(name, dt, q, k, v, o, lse, scale, causal, stream, want_lse,
+                out_dtype=torch.float32)
 
 
 def _decode(fname, dtype, q, kcache, vcache, seqlens, Hkv, o, lse, scale, stream, want_lse,
@@ -254,17 +275,19 @@ def attn_merge(o_acc, lse_acc, o_part, lse_part, o_out=None, stream=None) -> Non
     """Fold a partial result (o_part, lse_part) into the fp32 accumulator in place.
 
     o_acc float32 [..., d] and lse_acc float32 [...] (same leading shape as
-    o_part / lse_part); o_part bf16 or fp16; o_out (optional, o_part's dtype
-    and shape) also receives the merged O rounded. A row with lse_acc = -inf is
-    empty (o_acc not read). Runs ``attn_merge`` / ``attn_merge_f16``.
+    o_part / lse_part); o_part bf16, fp16 or float32 (an unrounded partial from
+    ``attn_fwd_partial``); o_out (optional, o_part's shape; bf16 or fp16, o_part's
+    dtype unless o_part is float32) also receives the merged O rounded. A row
+    with lse_acc = -inf is empty (o_acc not read). Runs ``attn_merge`` /
+    ``attn_merge_f16``, or ``attn_merge_partial`` / ``attn_merge_partial_f16``.
     """
     import torch
 
     for t, n in ((o_acc, "o_acc"), (lse_acc, "lse_acc"), (o_part, "o_part"),
                  (lse_part, "lse_part")):
         _dev(t, n)
-    if o_part.dtype not in (torch.bfloat16, torch.float16):
-        raise ValueError("o_part must be bf16 or fp16")
+    if o_part.dtype not in (torch.bfloat16, torch.float16, torch.float32):
+        raise ValueError("o_part must be bf16, fp16 or float32")
     if o_acc.dtype != torch.float32 or lse_acc.dtype != torch.float32 or \
             lse_part.dtype != torch.float32:
         raise ValueError("o_acc, lse_acc and lse_part must be float32")
@@ -275,9 +298,16 @@ def attn_merge(o_acc, lse_acc, o_part, lse_part, o_out=None, stream=None) -> Non
         raise ValueError("o_acc, lse_acc, o_part and lse_part shapes disagree")
     if o_out is not None:
         _dev(o_out, "o_out")
-        if o_out.dtype != o_part.dtype or tuple(o_out.shape) != tuple(o_part.shape):
-            raise ValueError("o_out must match o_part")
-    name = "attn_merge_f16" if o_part.dtype == torch.float16 else "attn_merge"
+        if tuple(o_out.shape) != tuple(o_part.shape) or (
+                o_out.dtype != o_part.dtype if o_part.dtype != torch.float32
+                else o_out.dtype not in (torch.bfloat16, torch.float16)):
+            raise ValueError("o_out must match o_part's shape (and dtype, or bf16 / fp16 "
+                             "for a float32 o_part)")
+    if o_part.dtype == torch.float32:
+        f16 = o_out is not None and o_out.dtype == torch.float16
+        name = "attn_merge_partial_f16" if f16 else "attn_merge_partial"
+    else:
+        name = "attn_merge_f16" if o_part.dtype == torch.float16 else "attn_merge"
     rows = o_part.numel() // d if d else 0
     with _on_device(o_acc, lse_acc, o_part, lse_part, o_out):
         code = getattr(load_library(), name)(

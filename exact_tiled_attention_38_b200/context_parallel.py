@@ -150,15 +150,13 @@ class LocalRing:
 
 
 class CudaOps:
-    """The library's kernels: prefill on one chunk pair, and the LSE merge."""
+    """The library's kernels: prefill on one chunk pair with O kept in float32,
+    and the LSE merge of such a partial into the running accumulator."""
 
     def attention(self, q, k, v, scale, causal, o, lse):
-        import torch
+        from . import attn_fwd_partial
 
-        from . import attn_fwd, attn_fwd_f16
-
-        fn = attn_fwd_f16 if q.dtype == torch.float16 else attn_fwd
-        return fn(q, k, v, o=o, lse=lse, scale=scale, causal=causal)
+        return attn_fwd_partial(q, k, v, o=o, lse=lse, scale=scale, causal=causal)
 
     def merge(self, o_acc, lse_acc, o_part, lse_part, o_out):
         from . import attn_merge
@@ -196,7 +194,10 @@ def ring_attention(q, k, v, causal: bool = True, scale: Optional[float] = None,
     o = torch.empty_like(q)
     o_acc = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     lse_acc = torch.full(q.shape[:-1], float("-inf"), dtype=torch.float32, device=q.device)
-    part_o = torch.empty_like(q[0])
+    # Every partial O stays unrounded (float32; wider inputs keep their own
+    # type), so the 2W - 1 folds of a query chunk round its output once.
+    part_dt = torch.float32 if q.dtype in (torch.bfloat16, torch.float16) else q.dtype
+    part_o = torch.empty(q.shape[1:], dtype=part_dt, device=q.device)
     part_lse = torch.empty(q.shape[1:-1], dtype=torch.float32, device=q.device)
     cur_k, cur_v = k, v
     nxt_k, nxt_v = (torch.empty_like(k), torch.empty_like(v)) if world > 1 else (None, None)

@@ -5,7 +5,7 @@
 //   decode_sm100.cuh     decode split pass on CUDA cores (d = 64, groups <= 4)
 //                        and the LSE combine
 //   decode_ps_sm100.cuh  decode as one persistent streaming pass on tcgen05
-//                        (d = 128, groups 8..32): plan, stream, gather
+//                        (d = 128, groups 2..32): plan, stream, gather
 //   decode_tc_sm100.cuh  helpers of the tcgen05 decode (and its earlier
 //                        one-CTA-per-split pass, kept as a knob)
 //   generic_fwd.cuh      prefill and decode for the other head sizes
@@ -17,6 +17,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/attn.h"
 #include "decode_ps_sm100.cuh"
@@ -149,13 +150,13 @@ inline bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
 inline bool tensor_core_d(int d) { return d == 64 || d == 128; }
 inline bool generic_d(int d) { return d >= 8 && d <= generic::kMaxD && d % 8 == 0; }
 
-template <typename T>
+template <typename T, bool OUT_F32 = false>
 int launch_generic(generic::GParams p, int BH, int Nq, cudaStream_t st) {
   p.BH = BH;
   const int ny = BH < generic::kGridY ? BH : generic::kGridY;
   const dim3 grid((Nq + generic::kRows - 1) / generic::kRows, ny,
                   (BH + generic::kGridY - 1) / generic::kGridY);
-  generic::attn_generic_kernel<T>
+  generic::attn_generic_kernel<T, OUT_F32>
       <<<grid, generic::kThreads, generic::smem_bytes(p.d), st>>>(p);
   return launch_status();
 }
@@ -176,6 +177,24 @@ int encode_3d(CUtensorMap* map, const void* base, bool bf16, int D, long long ro
                         3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// 3-D map over a [Z][rows][D] fp32 tensor, box 32 x 32 x 1 (128-byte rows),
+// 128-byte swizzle; used for stores of unrounded partial outputs.
+int encode_3d_f32(CUtensorMap* map, const void* base, int D, long long rows, long long Z) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return ATTN_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(Z)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4,
+                                 static_cast<cuuint64_t>(rows) * D * 4};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -226,12 +245,12 @@ int launch_fill_empty(void* o, float* lse, long long rows, int D, cudaStream_t s
 #define ETA_PREFILL_SPLIT 1
 #endif
 
-template <int D, typename T, bool CAUSAL, bool WINDOW = false>
+template <int D, typename T, bool CAUSAL, bool WINDOW = false, bool OUT_F32 = false>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& to, const prefill::Params& p, int grid, cudaStream_t st) {
   constexpr int SPLIT = D == 128 ? ETA_PREFILL_SPLIT : 1;
   auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, WINDOW, ETA_PREFILL_POLY8, false, SPLIT,
-                                           ETA_PREFILL_PREFETCH_Q != 0>;
+                                           ETA_PREFILL_PREFETCH_Q != 0, OUT_F32>;
   constexpr int smem = prefill::Cfg<D>::kSmemBytes;
   static PerDeviceOnce attr;
   const cudaError_t attr_err = attr.run([&]() {
@@ -242,7 +261,8 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   return launch_status();
 }
 
-template <typename T>
+// OUT_F32: o is float32 (the unrounded O of a partial result), else T.
+template <typename T, bool OUT_F32 = false>
 int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
         int Nq, int Nk, int d, float scale, int causal, cudaStream_t st, uint64_t wait_ns,
         int debug_flags, int window = 0) {
@@ -261,7 +281,10 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   DeviceInfo info;
   if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
   if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
-  if (Nk == 0) return launch_fill_empty<T>(o, lse, static_cast<long long>(B) * Hq * Nq, d, st);
+  if (Nk == 0) {
+    using TO = typename std::conditional<OUT_F32, float, T>::type;
+    return launch_fill_empty<TO>(o, lse, static_cast<long long>(B) * Hq * Nq, d, st);
+  }
   if (!tensor_core_d(d)) {
     generic::GParams g;
     g.q = q;
@@ -280,13 +303,15 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     g.window = window;
     g.scale_log2 = scale * 1.4426950408889634f;
     g.seqlens = nullptr;
-    return launch_generic<T>(g, B * Hq, Nq, st);
+    return launch_generic<T, OUT_F32>(g, B * Hq, Nq, st);
   }
 
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap tq, tk, tv, to;
   int rc = encode_3d(&tq, q, bf16, d, Nq, static_cast<long long>(B) * Hq);
-  if (rc == ATTN_OK) rc = encode_3d(&to, o, bf16, d, Nq, static_cast<long long>(B) * Hq, 32);
+  if (rc == ATTN_OK)
+    rc = OUT_F32 ? encode_3d_f32(&to, o, d, Nq, static_cast<long long>(B) * Hq)
+                 : encode_3d(&to, o, bf16, d, Nq, static_cast<long long>(B) * Hq, 32);
   if (rc == ATTN_OK) rc = encode_3d(&tk, k, bf16, d, Nk, static_cast<long long>(B) * Hkv);
   if (rc == ATTN_OK) rc = encode_3d(&tv, v, bf16, d, Nk, static_cast<long long>(B) * Hkv);
   if (rc != ATTN_OK) return rc;
@@ -310,6 +335,14 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   p.debug_flags = debug_flags;
   p.window = window;
   const int grid = static_cast<int>(total < info.sm_count ? total : info.sm_count);
+  if constexpr (OUT_F32) {
+    if (window > 0) return ATTN_ERR_INVALID;
+    if (d == 128)
+      return causal ? launch_prefill<128, T, true, false, true>(tq, tk, tv, to, p, grid, st)
+                    : launch_prefill<128, T, false, false, true>(tq, tk, tv, to, p, grid, st);
+    return causal ? launch_prefill<64, T, true, false, true>(tq, tk, tv, to, p, grid, st)
+                  : launch_prefill<64, T, false, false, true>(tq, tk, tv, to, p, grid, st);
+  }
   if (window > 0)
     return d == 128 ? launch_prefill<128, T, true, true>(tq, tk, tv, to, p, grid, st)
                     : launch_prefill<64, T, true, true>(tq, tk, tv, to, p, grid, st);
@@ -363,6 +396,11 @@ inline int decode_group_tile(int G) { return (G <= 4 || ETA_DECODE_MAX_GP == 4) 
 #ifndef ETA_DECODE_PS_MIN_G
 #define ETA_DECODE_PS_MIN_G 2
 #endif
+// Softmax warps per key quarter in the persistent pass for groups of 17 to 32
+// heads: 2 (each thread takes 16 of the heads of its key) or 1.
+#ifndef ETA_DECODE_PS_HS32
+#define ETA_DECODE_PS_HS32 2
+#endif
 inline bool decode_use_ps(int G, int d) {
   return ETA_DECODE_PS_MIN_G > 0 && d == 128 && G >= ETA_DECODE_PS_MIN_G && G <= 32;
 }
@@ -374,19 +412,21 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Device workspace of the persistent pass, byte offsets: the plan (token
 // offsets int64 [B], tile offsets int32 [B + 1]) and, when CTAs take equal
-// tile ranges, the partials of segments cut between CTAs (slot segment + cta:
-// B * Hkv + nc - 1 slots of G rows).
+// tile ranges, each CTA's first tile (int4 [nc]) and the partials of segments
+// cut between CTAs (slot segment + cta: B * Hkv + nc - 1 slots of G rows).
 struct PsLayout {
-  size_t tok_off, tile_off, part_o, part_lse, total;
+  size_t tok_off, tile_off, starts, part_o, part_lse, total;
 };
 inline PsLayout ps_layout(int B, int Hkv, int G, int nc, bool partials) {
   PsLayout L;
   L.tok_off = 0;
   L.tile_off = align_up(static_cast<size_t>(B) * 8, 256);
   size_t end = L.tile_off + (static_cast<size_t>(B) + 1) * 4;
-  L.part_o = L.part_lse = 0;
+  L.starts = L.part_o = L.part_lse = 0;
   if (partials) {
     const size_t slots = static_cast<size_t>(B) * Hkv + nc - 1;
+    L.starts = align_up(end, 256);
+    end = L.starts + static_cast<size_t>(nc) * 16;
     L.part_o = align_up(end, 256);
     end = L.part_o + slots * G * decode_ps::D * 4;
     L.part_lse = align_up(end, 256);
@@ -446,25 +486,24 @@ int launch_decode_tc(const decode::DParams& p, cudaStream_t st) {
 }
 
 // Plan, persistent stream and gather of the d = 128 decode; `ws` holds the
-// layout `L`. seg_aligned: whole segments per CTA (L has no partials).
-template <int NP, int GP, typename T>
+// layout `L`. seg_aligned: whole segments per CTA (L has no partials, and
+// there is nothing to gather).
+template <int NP, int GP, int HS, typename T>
 int launch_decode_ps(const CUtensorMap& tq, decode_ps::PParams p, const PsLayout& L, char* ws,
                      int nc, cudaStream_t st) {
-  auto kern = decode_ps::attn_decode_persistent_kernel<NP, GP, T>;
+  auto kern = decode_ps::attn_decode_persistent_kernel<NP, GP, HS, T>;
   constexpr int smem = decode_ps::PCfg<NP>::kSmemBytes;
   static PerDeviceOnce attr;
   const cudaError_t attr_err = attr.run([&]() {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err);
-  long long* tok_off = reinterpret_cast<long long*>(ws + L.tok_off);
-  int* tile_off = reinterpret_cast<int*>(ws + L.tile_off);
-  p.tok_off = tok_off;
-  p.tile_off = tile_off;
+  p.tok_off = reinterpret_cast<long long*>(ws + L.tok_off);
+  p.tile_off = reinterpret_cast<int*>(ws + L.tile_off);
+  p.starts = L.starts ? reinterpret_cast<int4*>(ws + L.starts) : nullptr;
   p.part_o = L.part_o ? reinterpret_cast<float*>(ws + L.part_o) : nullptr;
   p.part_lse = L.part_lse ? reinterpret_cast<float*>(ws + L.part_lse) : nullptr;
-  decode_ps::attn_decode_plan_kernel<<<1, decode_ps::kPlanThreads, 0, st>>>(
-      p.seqlens, tok_off, tile_off, p.B, p.Hkv, p.window);
+  decode_ps::attn_decode_plan_kernel<<<1, decode_ps::kPlanThreads, 0, st>>>(p, nc);
   int rc = launch_status();
   if (rc != ATTN_OK) return rc;
   // The stream and gather kernels are launched as programmatic dependents:
@@ -475,13 +514,14 @@ int launch_decode_ps(const CUtensorMap& tq, decode_ps::PParams p, const PsLayout
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(nc));
-  cfg.blockDim = dim3(decode_ps::kThreads);
+  cfg.blockDim = dim3(decode_ps::Roles<HS>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, p);
   if (e != cudaSuccess) return cuda_fail(e);
+  if (p.seg_aligned) return launch_status();  // no cut segments, nothing to gather
   const long long rows = static_cast<long long>(p.B) * p.Hq;
   cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
   cfg.blockDim = dim3(128);
@@ -521,10 +561,10 @@ int decode_ps_run(const void* q, const void* kc, const void* vc, const int32_t* 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
   const PsLayout L = ps_layout(B, Hkv, G, nc, !seg_aligned);
-  if (G <= 4) return launch_decode_ps<16, 4, T>(tq, p, L, ws, nc, st);
-  if (G <= 8) return launch_decode_ps<16, 8, T>(tq, p, L, ws, nc, st);
-  if (G <= 16) return launch_decode_ps<16, 16, T>(tq, p, L, ws, nc, st);
-  return launch_decode_ps<32, 32, T>(tq, p, L, ws, nc, st);
+  if (G <= 4) return launch_decode_ps<16, 4, 1, T>(tq, p, L, ws, nc, st);
+  if (G <= 8) return launch_decode_ps<16, 8, 1, T>(tq, p, L, ws, nc, st);
+  if (G <= 16) return launch_decode_ps<16, 16, 1, T>(tq, p, L, ws, nc, st);
+  return launch_decode_ps<32, 32, ETA_DECODE_PS_HS32, T>(tq, p, L, ws, nc, st);
 }
 
 template <int D, typename T>
@@ -660,7 +700,8 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
 namespace eta {
 namespace api {
 
-template <typename T>
+// T: type of o_out; TP: type of o_part (T, or float for unrounded partials).
+template <typename T, typename TP = T>
 int merge_run(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
               void* o_out, long long rows, int d, cudaStream_t st) {
   if (rows < 0 || !generic_d(d)) return rows < 0 ? ATTN_ERR_INVALID : ATTN_ERR_UNSUPPORTED;
@@ -678,8 +719,8 @@ int merge_run(float* o_acc, float* lse_acc, const void* o_part, const float* lse
   const long long want = (rows + rows_per_block - 1) / rows_per_block;
   const long long cap = 8LL * info.sm_count;  // grid-stride beyond 8 blocks per SM
   const int blocks = static_cast<int>(want < cap ? want : cap);
-  merge::attn_merge_kernel<T><<<blocks, merge::kThreads, 0, st>>>(
-      o_acc, lse_acc, reinterpret_cast<const T*>(o_part), lse_part, reinterpret_cast<T*>(o_out),
+  merge::attn_merge_kernel<T, TP><<<blocks, merge::kThreads, 0, st>>>(
+      o_acc, lse_acc, reinterpret_cast<const TP*>(o_part), lse_part, reinterpret_cast<T*>(o_out),
       rows, d);
   return launch_status();
 }
@@ -809,6 +850,35 @@ int attn_merge_f16(float* o_acc, float* lse_acc, const void* o_part, const float
                    void* o_out, long long rows, int d, attn_stream_t stream) {
   return eta::api::merge_run<__half>(o_acc, lse_acc, o_part, lse_part, o_out, rows, d,
                                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_partial(const void* q, const void* k, const void* v, float* o, float* lse, int B,
+                     int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                     attn_stream_t stream) {
+  return eta::api::fwd<__nv_bfloat16, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                                            reinterpret_cast<cudaStream_t>(stream),
+                                            eta::kDefaultWaitNs, 0);
+}
+
+int attn_fwd_partial_f16(const void* q, const void* k, const void* v, float* o, float* lse, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                         attn_stream_t stream) {
+  return eta::api::fwd<__half, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                                     reinterpret_cast<cudaStream_t>(stream), eta::kDefaultWaitNs,
+                                     0);
+}
+
+int attn_merge_partial(float* o_acc, float* lse_acc, const float* o_part, const float* lse_part,
+                       void* o_out, long long rows, int d, attn_stream_t stream) {
+  return eta::api::merge_run<__nv_bfloat16, float>(o_acc, lse_acc, o_part, lse_part, o_out, rows,
+                                                   d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_merge_partial_f16(float* o_acc, float* lse_acc, const float* o_part,
+                           const float* lse_part, void* o_out, long long rows, int d,
+                           attn_stream_t stream) {
+  return eta::api::merge_run<__half, float>(o_acc, lse_acc, o_part, lse_part, o_out, rows, d,
+                                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, float* lse, int B,

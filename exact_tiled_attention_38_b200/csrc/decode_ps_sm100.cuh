@@ -18,11 +18,13 @@
 //   attn_decode_plan_kernel        one CTA: per sequence, token offset in the
 //                                  packed cache (int64) and tile offset in the
 //                                  global tile order (int32 prefix over
-//                                  sequences, KV heads included)
+//                                  sequences, KV heads included); each CTA's
+//                                  first tile position; O = 0, LSE = -inf for
+//                                  empty sequences
 //   attn_decode_persistent_kernel  the stream (below)
-//   attn_decode_gather_kernel      one warp per (sequence, query head): merges
-//                                  the partials of segments cut between CTAs,
-//                                  writes O = 0, LSE = -inf for empty ones
+//   attn_decode_gather_kernel      one warp per (sequence, query head) of a
+//                                  segment cut between CTAs: merges its
+//                                  partials by their log-sum-exp
 //
 // Per tile (G query heads of KV head g, padded to NP = 16 or 32):
 //   S^T = K_j Q^T      M = 128 keys, N = NP, K = 128 dims; A = K tile
@@ -60,10 +62,19 @@ namespace decode_ps {
 constexpr int D = 128;
 constexpr int TK = 128;  // keys per tile
 constexpr int kStages = 3;
-constexpr int kSoftWarps = 4;
-constexpr int kMmaWarp = 4;
-constexpr int kProdWarp0 = 5;
-constexpr int kThreads = 32 * (kProdWarp0 + kStages);
+constexpr int kSoftWarps = 4;  // key quarters of a tile (tensor-memory lane quarters)
+
+// Warp roles for HS softmax warps per key quarter (HS = 2: the two warps of a
+// quarter split the heads of its keys): softmax warps 0 .. 4 HS - 1, then the
+// MMA warp, then one producer warp per ring stage.
+template <int HS>
+struct Roles {
+  static constexpr int kSoft = kSoftWarps * HS;
+  static constexpr int kMma = kSoft;
+  static constexpr int kProd0 = kSoft + 1;
+  static constexpr int kThreads = 32 * (kProd0 + kStages);
+};
+constexpr int kThreads = Roles<1>::kThreads;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kTmemCols = 128;
 constexpr int kPlanThreads = 1024;
@@ -91,6 +102,7 @@ struct PParams {
   float* lse;                // [B][Hq] natural log, or NULL
   float* part_o;             // [slots][G][D]: normalised partial O of a cut segment
   float* part_lse;           // [slots][G]: its log-sum-exp, log2 units
+  int4* starts;              // [nc]: (b, g, i) of each CTA's first tile (equal tile ranges)
   int B;
   int Hq;
   int Hkv;
@@ -119,10 +131,11 @@ __device__ __forceinline__ int first_key(int len, int window) {
 // Exclusive prefix sums over the B sequences (one CTA): token offsets of the
 // packed cache and tile offsets of the global tile order (Hkv segments of
 // ceil(keys read / 128) tiles per sequence). tile_off[B] is the total.
-__global__ void __launch_bounds__(kPlanThreads) attn_decode_plan_kernel(const int* __restrict__ seqlens,
-                                                                      long long* __restrict__ tok_off,
-                                                                      int* __restrict__ tile_off,
-                                                                      int B, int Hkv, int window) {
+__global__ void __launch_bounds__(kPlanThreads) attn_decode_plan_kernel(const PParams p, int nc) {
+  const int* __restrict__ seqlens = p.seqlens;
+  long long* __restrict__ tok_off = const_cast<long long*>(p.tok_off);
+  int* __restrict__ tile_off = const_cast<int*>(p.tile_off);
+  const int B = p.B, Hkv = p.Hkv, window = p.window;
   __shared__ long long s_tok[kPlanThreads / 32];
   __shared__ long long s_til[kPlanThreads / 32];
   griddep_launch_dependents();  // the stream kernel may start its set-up now
@@ -169,14 +182,35 @@ __global__ void __launch_bounds__(kPlanThreads) attn_decode_plan_kernel(const in
   __syncthreads();
   long long t_run = xt - tok + (warp > 0 ? s_tok[warp - 1] : 0);  // exclusive
   long long l_run = xl - til + (warp > 0 ? s_til[warp - 1] : 0);
+  const long long T = s_til[31];  // all tiles
   for (int b = b0; b < b1; ++b) {
     const int len = max(seqlens[b], 0);
+    const int nt = (len - first_key(len, window) + TK - 1) / TK;
     tok_off[b] = t_run;
     tile_off[b] = static_cast<int>(l_run);
+    if (nt == 0) {
+      // An empty sequence: no CTA visits it. O = 0, LSE = -inf.
+      for (int h = 0; h < p.Hq; ++h) {
+        const size_t row = static_cast<size_t>(b) * p.Hq + h;
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) + row * D);
+        for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (p.lse != nullptr) p.lse[row] = -INFINITY;
+      }
+    } else if (!p.seg_aligned) {
+      // CTAs of the equal tile ranges whose first tile lies in this sequence:
+      // CTA c starts at tile c * T / nc.
+      const long long span = static_cast<long long>(Hkv) * nt;
+      for (long long c = (l_run * nc + T - 1) / T; c < nc && c * T / nc < l_run + span; ++c) {
+        const long long lo = c * T / nc;
+        if (lo >= (c + 1) * T / nc) continue;  // an empty range: the CTA does nothing
+        const int r = static_cast<int>(lo - l_run);
+        p.starts[c] = make_int4(b, r / nt, r % nt, 0);
+      }
+    }
     t_run += len;
-    l_run += static_cast<long long>(Hkv) * ((len - first_key(len, window) + TK - 1) / TK);
+    l_run += static_cast<long long>(Hkv) * nt;
   }
-  if (threadIdx.x == kPlanThreads - 1) tile_off[B] = static_cast<int>(s_til[31]);
+  if (threadIdx.x == kPlanThreads - 1) tile_off[B] = static_cast<int>(T);
 }
 
 // Tile range [lo, hi) of CTA c of nc in the global tile order.
@@ -329,13 +363,17 @@ __device__ __forceinline__ void gather4(const float* red, float (&out)[GP], Op o
 }
 
 // NP: MMA width (the group padded to 16 or 32); GP <= NP: the heads the
-// softmax processes (the group padded to 4, 8, 16 or 32).
-template <int NP, int GP, typename T>
-__global__ void __launch_bounds__(kThreads, 1)
+// softmax processes (the group padded to 4, 8, 16 or 32); HS: softmax warps
+// per key quarter, each taking GP / HS of the heads.
+template <int NP, int GP, int HS, typename T>
+__global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     attn_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_q, const PParams p) {
   static_assert(GP == 4 || GP == 8 || GP == 16 || GP == 32, "softmax group");
   static_assert(GP <= NP && (GP > 16) == (NP == 32), "widths");
+  static_assert(HS == 1 || (HS == 2 && GP == 32), "head split");
   using C = PCfg<NP>;
+  using R = Roles<HS>;
+  constexpr int GPT = GP / HS;  // heads per softmax thread
   using decode_tc::sw128_off;
   using decode_tc::tmem_ld_np;
   using decode_tc::tmem_st_np;
@@ -371,8 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_ready[i], 1);
-      mbar_init(&p_ready[i], 32 * kSoftWarps);
-      mbar_init(&x_bar[i], 32 * kSoftWarps);
+      mbar_init(&p_ready[i], 32 * R::kSoft);
+      mbar_init(&x_bar[i], 32 * R::kSoft);
       mbar_init(&q_full[i], 1);
       mbar_init(&q_free[i], 1);
     }
@@ -382,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ctl->wait_ns = p.wait_ns;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == R::kMma) {
     tmem_alloc(tmem_holder, kTmemCols);
     tmem_relinquish();
     if (lane == 0) tma_prefetch_desc(&tm_q);
@@ -404,16 +442,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Range rg = cta_range(p, c, gridDim.x);
   const int n = rg.hi > rg.lo ? static_cast<int>(rg.hi - rg.lo) : 0;  // tiles of this CTA
   Cursor cur;
-  if (n > 0) cur.seek(p, rg.lo);
+  if (n > 0) {
+    if (p.seg_aligned) {
+      cur.seek(p, rg.lo);
+    } else {  // the plan found this CTA's first tile
+      const int4 st = p.starts[c];
+      cur.b = st.x;
+      cur.load_seq(p);
+      cur.g = st.y;
+      cur.i = st.z;
+    }
+  }
 
   if (n == 0) {
     // no tiles for this CTA (uniform over the CTA)
-  } else if (warp >= kProdWarp0) {
+  } else if (warp >= R::kProd0) {
     // ------------------------------------------------------------ producers
     // Producer pw fills stage pw with the CTA's tiles pw, pw + 3, ... Lane l
     // copies 16-byte unit (l % 16) of rows 2i + l / 16: each instruction reads
     // two whole 256-byte cache rows.
-    const int pw = warp - kProdWarp0;
+    const int pw = warp - R::kProd0;
     bool ok = true;
     const uint32_t kdst = smem_u32(smem + pw * C::kStageBytes);
     const uint32_t vdst = kdst + C::kTileBytes;
@@ -444,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int a = 0; a < kStages && j + 1 + a < n; ++a) cur.next(p);
     }
     cp_async_wait_all();  // no copy may land after the CTA exits
-  } else if (warp == kMmaWarp) {
+  } else if (warp == R::kMma) {
     // ------------------------------------------------------------ MMA issue and Q loads
     constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
     constexpr uint32_t idesc_s = umma_idesc_f16(fmt, TK, NP, 0, 0);
@@ -551,21 +599,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (nq[buf] > 0) drain_bar(&q_full[buf], (nq[buf] - 1) & 1, ctl, kSiteDrain);
   } else {
     // ------------------------------------------------------------ softmax and epilogue
-    // Each thread holds the GP (>= G) head scores of its key. The padded rows
-    // GP..NP-1 of both P^T buffers are zeroed once here and never written
-    // again, so the products' padded columns stay zero.
-    const int krow = warp * 32 + lane;  // this thread's key in a tile (tensor-memory lane)
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // Warp w owns the keys of quarter q4 = w % 4 (tensor-memory lanes 32 q4 ..
+    // 32 q4 + 31) and heads hh GPT .. hh GPT + GPT - 1, hh = w / 4; each
+    // thread holds its key's scores of those heads. The padded rows GP..NP-1
+    // of both P^T buffers are zeroed once here and never written again, so
+    // the products' padded columns stay zero.
+    const int q4 = warp & 3;
+    const int hh = warp >> 2;
+    const int h0 = hh * GPT;                  // first head of this thread
+    const int krow = q4 * 32 + lane;          // this thread's key in a tile (tensor-memory lane)
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const float sl2 = p.scale_log2;
     if constexpr (GP < NP) {
-      for (int i = threadIdx.x; i < 2 * 2 * (NP - GP) * 8; i += 32 * kSoftWarps) {
+      for (int i = threadIdx.x; i < 2 * 2 * (NP - GP) * 8; i += 32 * R::kSoft) {
         const int chunk = i & 7, row = GP + ((i >> 3) % (NP - GP)), box = i / (8 * (NP - GP));
         *reinterpret_cast<uint4*>(sP + box * C::kQBox + row * 128 + chunk * 16) =
             make_uint4(0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();
     }
-    float m[GP], l[GP];
+    float m[GPT], l[GPT];
     bool ok = true;
     uint32_t xc = 0;        // uses of the x_bar / red exchange so far
     bool piece_whole = false;
@@ -575,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (first) {
         piece_whole = (cur.i == 0);
 #pragma unroll
-        for (int h = 0; h < GP; ++h) {
+        for (int h = 0; h < GPT; ++h) {
           m[h] = -INFINITY;
           l[h] = 0.f;
         }
@@ -583,29 +636,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (last) piece_whole = piece_whole && (cur.i == cur.nt - 1);
       if (!(ok = decode::warp_all_d(wait_bar(&s_ready[j & 1], (j >> 1) & 1, ctl, kSiteS)))) break;
       tc_fence_after();
-      uint32_t r[NP];
-      tmem_ld_np<NP>(tS0 + lane_off + (j & 1) * NP, r);
+      uint32_t r[GPT < 16 ? 16 : GPT];
+      tmem_ld_np<(GPT < 16 ? 16 : GPT)>(tS0 + lane_off + (j & 1) * NP + h0, r);
       const bool valid = cur.k0 + cur.i * TK + krow < cur.len;
-      float s[GP], wm[GP];
+      float s[GPT], wm[GPT];
 #pragma unroll
-      for (int h = 0; h < GP; ++h) {
-        s[h] = (valid && h < G) ? __uint_as_float(r[h]) * sl2 : -INFINITY;
+      for (int h = 0; h < GPT; ++h) {
+        s[h] = (valid && h0 + h < G) ? __uint_as_float(r[h]) * sl2 : -INFINITY;
         wm[h] = s[h];
       }
       // tile max per head: this warp's 32 keys by a reduce-scatter (lane l ends
-      // with head l % GP), then the four warps through shared memory
-      const float wmax = reduce_scatter<GP>(wm, lane, MaxOp());
+      // with head h0 + l % GPT), then the four key quarters through shared memory
+      const float wmax = reduce_scatter<GPT>(wm, lane, MaxOp());
       float* rb = red + (xc & 1) * (kSoftWarps * NP);
-      if (lane < GP) rb[warp * NP + lane] = wmax;
+      if (lane < GPT) rb[q4 * NP + h0 + lane] = wmax;
       mbar_arrive(&x_bar[xc & 1]);
       if (!(ok = decode::warp_all_d(wait_bar(&x_bar[xc & 1], (xc >> 1) & 1, ctl, kSiteX)))) break;
       ++xc;
-      float tm[GP];
-      gather4<GP, NP>(rb, tm, MaxOp());
-      float alpha[GP];
+      float tm[GPT];
+      gather4<GPT, NP>(rb + h0, tm, MaxOp());
+      float alpha[GPT];
       bool rescale = false;
 #pragma unroll
-      for (int h = 0; h < GP; ++h) {
+      for (int h = 0; h < GPT; ++h) {
         alpha[h] = 1.f;
         if (tm[h] > m[h] + kRescaleThreshold) {
           alpha[h] = ex2_approx(m[h] - tm[h]);  // m = -inf gives 0
@@ -616,14 +669,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (rescale && !first) {
         // O^T was last written by PV(j-1) of this piece; wait for it, then
-        // scale this warp's 32 dims by the heads' alpha.
+        // scale this warp's 32 dims of its heads by their alpha.
         if (!(ok = decode::warp_all_d(wait_bar(pv_done, (j - 1) & 1, ctl, kSitePv)))) break;
         tc_fence_after();
-        uint32_t o[NP];
-        tmem_ld_np<NP>(tO + lane_off, o);
+        uint32_t o[GPT < 16 ? 16 : GPT];
+        tmem_ld_np<(GPT < 16 ? 16 : GPT)>(tO + lane_off + h0, o);
 #pragma unroll
-        for (int h = 0; h < GP; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-        tmem_st_np<NP>(tO + lane_off, o);
+        for (int h = 0; h < GPT; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+        tmem_st_np<(GPT < 16 ? 16 : GPT)>(tO + lane_off + h0, o);
         tmem_wait_st();
       }
       // P^T(j): row h, key krow, in buffer j % 2 (read by PV(j - 2), which
@@ -631,13 +684,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* pb = sP + (j & 1) * C::kPBuf + (krow >> 6) * C::kQBox;
       const int kc = krow & 63;
 #pragma unroll
-      for (int h = 0; h < GP; ++h) {
+      for (int h = 0; h < GPT; ++h) {
         float pv = 0.f;
-        if (h < G) {
+        if (h0 + h < G) {
           pv = ex2_approx(s[h] - (m[h] == -INFINITY ? 0.f : m[h]));
           l[h] += pv;
         }
-        *reinterpret_cast<uint16_t*>(pb + h * 128 + ((((kc >> 3) ^ (h & 7))) << 4) +
+        const int hr = h0 + h;
+        *reinterpret_cast<uint16_t*>(pb + hr * 128 + ((((kc >> 3) ^ (hr & 7))) << 4) +
                                      ((kc & 7) << 1)) = to_bits<T>(pv);
       }
       fence_proxy_async_smem();
@@ -646,37 +700,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (last) {
         // ---- end of a piece: row sums over the tile's 128 key slots, then O.
-        float lt[GP];
+        float lt[GPT];
 #pragma unroll
-        for (int h = 0; h < GP; ++h) lt[h] = l[h];
-        const float wsum = reduce_scatter<GP>(lt, lane, AddOp());
+        for (int h = 0; h < GPT; ++h) lt[h] = l[h];
+        const float wsum = reduce_scatter<GPT>(lt, lane, AddOp());
         float* rl = red + (xc & 1) * (kSoftWarps * NP);
-        if (lane < GP) rl[warp * NP + lane] = wsum;
+        if (lane < GPT) rl[q4 * NP + h0 + lane] = wsum;
         mbar_arrive(&x_bar[xc & 1]);
         if (!(ok = decode::warp_all_d(wait_bar(&x_bar[xc & 1], (xc >> 1) & 1, ctl, kSiteX)))) break;
         ++xc;
-        float tot[GP];
-        gather4<GP, NP>(rl, tot, AddOp());
+        float tot[GPT];
+        gather4<GPT, NP>(rl + h0, tot, AddOp());
         if (!(ok = decode::warp_all_d(wait_bar(pv_done, j & 1, ctl, kSitePv)))) break;
         tc_fence_after();
-        uint32_t o[NP];
-        tmem_ld_np<NP>(tO + lane_off, o);
+        uint32_t o[GPT < 16 ? 16 : GPT];
+        tmem_ld_np<(GPT < 16 ? 16 : GPT)>(tO + lane_off + h0, o);
         const int dim = krow;  // O^T lane = output dimension
         const int seg = cur.segment(p);
         const size_t row0 = static_cast<size_t>(cur.b) * p.Hq + static_cast<size_t>(cur.g) * G;
 #pragma unroll
-        for (int h = 0; h < GP; ++h) {
-          if (h < G) {
+        for (int h = 0; h < GPT; ++h) {
+          const int hg = h0 + h;
+          if (hg < G) {
             const float ov = tot[h] > 0.f ? __uint_as_float(o[h]) / tot[h] : 0.f;
             const float l2 = tot[h] > 0.f ? m[h] + lg2_approx(tot[h]) : -INFINITY;
             if (piece_whole) {
               // The whole segment lay in this CTA: this is the result.
-              reinterpret_cast<uint16_t*>(p.o)[(row0 + h) * D + dim] = to_bits<T>(ov);
-              if (dim == h && p.lse != nullptr) p.lse[row0 + h] = l2 * 0.69314718055994531f;
+              reinterpret_cast<uint16_t*>(p.o)[(row0 + hg) * D + dim] = to_bits<T>(ov);
+              if (dim == hg && p.lse != nullptr) p.lse[row0 + hg] = l2 * 0.69314718055994531f;
             } else {
               const size_t slot = static_cast<size_t>(seg) + c;
-              p.part_o[(slot * G + h) * D + dim] = ov;
-              if (dim == h) p.part_lse[slot * G + h] = l2;
+              p.part_o[(slot * G + hg) * D + dim] = ov;
+              if (dim == hg) p.part_lse[slot * G + hg] = l2;
             }
           }
         }
@@ -690,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == R::kMma) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -700,8 +755,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ gather
 // One warp per (sequence b, query head h): a segment cut between CTAs (in the
 // equal-tile-range mode) has one partial per CTA, in slots segment + cta;
-// merge them by their log-sum-exp. An empty sequence gets O = 0, LSE = -inf.
-// Segments that lay in one CTA were written by it and are skipped.
+// merge them by their log-sum-exp. Segments that lay in one CTA were written
+// by it, and empty sequences by the plan kernel; both are skipped.
 template <typename T>
 __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p, int nc) {
   griddep_wait();  // the stream kernel's partials and outputs are visible after this
@@ -713,16 +768,7 @@ __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p
   const int g = h / p.G;
   const int hh = h - g * p.G;
   const int nt = (p.tile_off[b + 1] - p.tile_off[b]) / p.Hkv;
-  T* dst = reinterpret_cast<T*>(p.o) + row * D + lane * 4;
-  if (nt == 0) {
-    uint2 z;
-    z.x = decode::pack2<T>(0.f, 0.f);
-    z.y = z.x;
-    *reinterpret_cast<uint2*>(dst) = z;
-    if (lane == 0 && p.lse != nullptr) p.lse[row] = -INFINITY;
-    return;
-  }
-  if (p.seg_aligned) return;
+  if (nt == 0 || p.seg_aligned) return;
   const long long T_all = p.tile_off[p.B];
   const long long a = p.tile_off[b] + static_cast<long long>(g) * nt;
   const int c0 = cta_of(a, T_all, nc);
@@ -754,7 +800,7 @@ __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p
   uint2 pk;
   pk.x = decode::pack2<T>(acc[0] * inv, acc[1] * inv);
   pk.y = decode::pack2<T>(acc[2] * inv, acc[3] * inv);
-  *reinterpret_cast<uint2*>(dst) = pk;
+  *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.o) + row * D + lane * 4) = pk;
   if (lane == 0 && p.lse != nullptr)
     p.lse[row] = tot > 0.f ? (mx + lg2_approx(tot)) * 0.69314718055994531f : -INFINITY;
 }

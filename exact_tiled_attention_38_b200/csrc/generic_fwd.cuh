@@ -121,7 +121,8 @@ __device__ __forceinline__ void visible_range(const GParams& p, int row, int& lo
   }
 }
 
-template <typename T>
+// OUT_F32: O is written as fp32 (not rounded), for partial results merged further.
+template <typename T, bool OUT_F32 = false>
 __global__ void __launch_bounds__(kThreads) attn_generic_kernel(const GParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int d = p.d;
@@ -258,7 +259,14 @@ __global__ void __launch_bounds__(kThreads) attn_generic_kernel(const GParams p)
     const int row = r0 + warp * kRowsPerWarp + i;
     if (row >= p.Nq) continue;
     const float inv = l[i] > 0.f ? 1.f / l[i] : 0.f;
-    if (lane < nchunk) {
+    if (OUT_F32 && lane < nchunk) {
+      float* dst = reinterpret_cast<float*>(p.o) + (static_cast<size_t>(bh) * p.Nq + row) * d +
+                   lane * 8;
+      *reinterpret_cast<float4*>(dst) =
+          make_float4(o[i][0] * inv, o[i][1] * inv, o[i][2] * inv, o[i][3] * inv);
+      *reinterpret_cast<float4*>(dst + 4) =
+          make_float4(o[i][4] * inv, o[i][5] * inv, o[i][6] * inv, o[i][7] * inv);
+    } else if (lane < nchunk) {
       uint4 w;
       w.x = pack_pair<T>(o[i][0] * inv, o[i][1] * inv);
       w.y = pack_pair<T>(o[i][2] * inv, o[i][3] * inv);

@@ -8,8 +8,8 @@
 // FlashAttention" ("Online Softmax") applied to whole key blocks; the decode
 // split combine is the same identity over many splits.
 //
-// attn_merge_kernel folds one partial (O_part in the input dtype, LSE_part
-// fp32) into an fp32 accumulator (o_acc, lse_acc) in place and optionally
+// attn_merge_kernel folds one partial (O_part in the input dtype or fp32,
+// LSE_part fp32) into an fp32 accumulator (o_acc, lse_acc) in place and optionally
 // writes the merged O rounded to the input dtype. A row whose accumulator LSE
 // is -inf is empty: its o_acc is not read. Each row is owned by the lanes of
 // one warp (8 columns per lane), so the row's LSE is read by all of them
@@ -64,10 +64,20 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <typename T>
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&f)[8]) {
+  const float4 x = *reinterpret_cast<const float4*>(p);
+  const float4 y = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+  f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
+}
+
+// T: type of the rounded output o_out; TP: type of the partial O (T, or fp32
+// for unrounded partials).
+template <typename T, typename TP = T>
 __global__ void __launch_bounds__(kThreads)
     attn_merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc,
-                      const T* __restrict__ o_part, const float* __restrict__ lse_part,
+                      const TP* __restrict__ o_part, const float* __restrict__ lse_part,
                       T* __restrict__ o_out, long long rows, int d) {
   const int cpr = d >> 3;          // 8-column chunks per row (1..32)
   const int rpw = 32 / cpr;        // rows per warp pass
@@ -108,7 +118,7 @@ __global__ void __launch_bounds__(kThreads)
         for (int e = 0; e < 8; ++e) a[e] = 0.f;
       }
       if (wp != 0.f) {
-        load8<T>(o_part + r * d + c * 8, pf);
+        load8<TP>(o_part + r * d + c * 8, pf);
       } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) pf[e] = 0.f;

@@ -30,6 +30,15 @@
 // P_t(j-1) occupied. The next item's Q loads and first S products overlap the
 // current item's epilogue.
 //
+// Head size 64 has room for P in tensor-memory columns of its own: per tile
+// S_t [256t, 256t+128), P_t [256t+128, 256t+192), O_t [256t+192, 256t+256).
+// The softmax then releases S_t (s_free) as soon as it has read it, and the
+// MMA thread issues S_t(j+1) at once, before P_t(j) V_j: the next scores are
+// ready when the softmax finishes a step, so the softmax groups run back to
+// back instead of waiting for the product chain. Before writing P_t (and
+// before rescaling O_t) the softmax waits for the previous P_t V product
+// (pv_done).
+//
 // Online softmax per row (fp32, log2 domain, c = scale * log2 e):
 //   m' = max over the tile of s * c; if m' > m + 8 the row's running max moves
 //   to m' and O and l are multiplied by 2^(m - m'); otherwise the stale max is
@@ -81,6 +90,8 @@ enum : unsigned {
   kSiteTurn = 9,
   kSiteXUp = 10,
   kSiteXDown = 11,
+  kSiteSFree = 12,
+  kSitePvDone = 13,
 };
 
 template <int D>
@@ -98,14 +109,25 @@ struct Cfg {
   static constexpr int kBarOff = kStgOff + 8 * kStgWarpBytes;
   // kv_full[S], kv_empty[S], then per tile: q_full, q_empty, s_ready, p_ready,
   // o_done, turn; then drain; then per row quarter of each tile the two
-  // exchange barriers of a split row (x_up: part 1 -> part 0, x_down: back).
-  static constexpr int kNumBars = 2 * kStages + 6 * NQT + 1 + 2 * 4 * NQT;
+  // exchange barriers of a split row (x_up: part 1 -> part 0, x_down: back);
+  // then per tile s_free and pv_done (P in columns of its own, D = 64).
+  static constexpr int kNumBars = 2 * kStages + 6 * NQT + 1 + 2 * 4 * NQT + 2 * NQT;
   static constexpr int kCtlOff = kBarOff + kNumBars * 8;
   // Row-statistics exchange between the two threads of a row (SPLIT = 2):
   // one float per query row of each tile.
   static constexpr int kXOff = kCtlOff + 64;
   static constexpr int kSmemBytes = kXOff + NQT * BM * 4 + 1024;  // + runtime 1024-byte alignment
+  // P in columns of its own (D = 64): S_t, P_t, O_t in 256 columns per tile.
+  static constexpr bool kOwnP = (D == 64);
   static constexpr uint32_t kOCol = 2 * BN;
+  __host__ __device__ static constexpr uint32_t s_col(int t) { return kOwnP ? 256u * t : BN * t; }
+  __host__ __device__ static constexpr uint32_t o_col(int t) {
+    return kOwnP ? 256u * t + BN + 64 : kOCol + D * t;
+  }
+  // first column of P_t (SPLIT = 1)
+  __host__ __device__ static constexpr uint32_t p_base(int t) {
+    return kOwnP ? 256u * t + BN : BN * t + kPCol;
+  }
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
@@ -306,8 +328,10 @@ __device__ __forceinline__ float exp_tile(const float (&s)[NC], float c, float m
   return (a0 + a1) + (b0 + b1);
 }
 
+// OUT_F32: O is written as fp32 (O / l, not rounded), for partial results
+// that are merged further (tm_o then maps an fp32 tensor with 32 x 32 boxes).
 template <int D, typename T, bool CAUSAL, bool WINDOW, int POLY8, bool PINGPONG, int SPLIT = 1,
-          bool PREFETCH_Q = false>
+          bool PREFETCH_Q = false, bool OUT_F32 = false>
 __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -337,6 +361,10 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
   uint64_t* drain = turn + NQT;
   uint64_t* x_up = drain + 1;        // [NQT * 4]
   uint64_t* x_down = x_up + 4 * NQT;  // [NQT * 4]
+  uint64_t* s_free = x_down + 4 * NQT;  // [NQT]: the softmax has read S_t (own-P layout)
+  uint64_t* pv_done = s_free + NQT;     // [NQT]: P_t V complete (own-P layout)
+  constexpr bool OWNP = C::kOwnP;
+  static_assert(!OWNP || (SPLIT == 1 && !PINGPONG), "own-P layout: one thread per row");
   CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem + C::kCtlOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kCtlOff + 32);
 
@@ -363,6 +391,10 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
     for (int i = 0; i < 4 * NQT; ++i) {
       mbar_init(&x_up[i], 32);
       mbar_init(&x_down[i], 32);
+    }
+    for (int t = 0; t < NQT; ++t) {
+      mbar_init(&s_free[t], 4 * 32 * SPLIT);
+      mbar_init(&pv_done[t], 1);
     }
     ctl->abort = 0;
     ctl->wait_ns = p.wait_ns;
@@ -461,51 +493,25 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
     uint32_t L = 0;
     int qi[NQT] = {0, 0};
     uint32_t pw[NQT] = {0, 0};
+    uint32_t sf[NQT] = {0, 0};  // score products issued per tile (own-P layout)
     bool ok = true;
     for (int r = 0; ok; ++r) {
       const int idx = item_index(r, cta, G);
       if (idx >= p.total) break;
       const Item it = decode_item<CAUSAL, WINDOW>(idx, p, nkv_all);
       const int nmax = max(it.n0, it.n1);
-      for (int j = 0; ok && j <= nmax; ++j) {
-        const uint32_t Lk = L + 2 * j;
-        const uint32_t Lv = L + 2 * j - 1;
-        bool have_k = false, have_v = false;
+      if constexpr (OWNP) {
+        // Own-P layout: per key tile j, first the score products S_t(j) (each
+        // as soon as the softmax has read S_t(j-1)), then P_t(j-1) V_{j-1}.
+        for (int j = 0; ok && j <= nmax; ++j) {
+          const uint32_t Lk = L + 2 * j;
+          const uint32_t Lv = L + 2 * j - 1;
+          bool have_k = false, have_v = false;
 #pragma unroll
-        for (int t = 0; t < NQT; ++t) {
-          if (!ok) break;
-          const int n = t ? it.n1 : it.n0;
-          const int s0 = t ? it.s1 : it.s0;  // this tile's first step
-          if (j >= 1 && j - 1 >= s0 && j - 1 < n) {
-            // O_t (+)= P_t(j-1) V_{j-1}. The p_ready arrival for an item's
-            // first step comes after the softmax group read O_t of its
-            // previous item, so O_t is free to be overwritten here.
-            if (!have_v) {
-              if (!(ok = warp_all(wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull))))
-                break;
-              have_v = true;
-            }
-            if (!(ok = warp_all(wait_bar(&p_ready[t], pw[t] & 1, ctl, kSitePReady)))) break;
-            ++pw[t];
-            tc_fence_after();
-            const uint32_t vd = v_lo + (((Lv % S) * C::kTileBytes) >> 4);
-            const uint32_t tS = tmem + t * BN;
-            const uint32_t tO = tmem + C::kOCol + t * D;
-            // P of keys 16kk..16kk+15: 8 columns. With SPLIT = 1 P fills columns
-            // [64, 128) of S_t; with SPLIT = 2 the two halves of the row sit at
-            // columns [0, 32) and [64, 96), each where its own thread read S.
-            // 16 keys = 16 rows of 128 bytes of V (2048 bytes = 128 in the address field)
-            if (j - 1 == s0)
-              umma_ts_w<0>(tO, tS + p_col<SPLIT>(0), desc_words(vd, d_hi), idesc_pv);
-            else
-              umma_ts_w<1>(tO, tS + p_col<SPLIT>(0), desc_words(vd, d_hi), idesc_pv);
-#pragma unroll
-            for (int kk = 1; kk < BN / 16; ++kk)
-              umma_ts_w<1>(tO, tS + p_col<SPLIT>(kk), desc_words(vd + kk * 128, d_hi), idesc_pv);
-            if (j - 1 == n - 1) umma_commit_w(&o_done[t]);
-          }
-          if (j >= s0 && j < n) {
-            // S_t = Q_t K_j^T
+          for (int t = 0; t < NQT; ++t) {
+            const int n = t ? it.n1 : it.n0;
+            const int s0 = t ? it.s1 : it.s0;
+            if (!ok || !(j >= s0 && j < n)) continue;
             if (!have_k) {
               if (!(ok = warp_all(wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull))))
                 break;
@@ -516,9 +522,14 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
               if (!(ok = warp_all(wait_bar(&q_full[t], qi[t] & 1, ctl, kSiteQFull)))) break;
               tc_fence_after();
             }
+            if (sf[t] > 0) {  // S_t's columns: the softmax has read the previous scores
+              if (!(ok = warp_all(wait_bar(&s_free[t], (sf[t] - 1) & 1, ctl, kSiteSFree)))) break;
+              tc_fence_after();
+            }
+            ++sf[t];
             const uint32_t kd = k_lo + (((Lk % S) * C::kTileBytes) >> 4);
             const uint32_t qd = q_lo + ((t * C::kTileBytes) >> 4);
-            const uint32_t tS = tmem + t * BN;
+            const uint32_t tS = tmem + C::s_col(t);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t koff = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
@@ -530,20 +541,122 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
             umma_commit_w(&s_ready[t]);
             if (j == n - 1) umma_commit_w(&q_empty[t]);
           }
+#pragma unroll
+          for (int t = 0; t < NQT; ++t) {
+            const int n = t ? it.n1 : it.n0;
+            const int s0 = t ? it.s1 : it.s0;
+            if (!ok || !(j >= 1 && j - 1 >= s0 && j - 1 < n)) continue;
+            if (!have_v) {
+              if (!(ok = warp_all(wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull))))
+                break;
+              have_v = true;
+            }
+            if (!(ok = warp_all(wait_bar(&p_ready[t], pw[t] & 1, ctl, kSitePReady)))) break;
+            ++pw[t];
+            tc_fence_after();
+            const uint32_t vd = v_lo + (((Lv % S) * C::kTileBytes) >> 4);
+            const uint32_t tP = tmem + C::p_base(t);
+            const uint32_t tO = tmem + C::o_col(t);
+            if (j - 1 == s0)
+              umma_ts_w<0>(tO, tP, desc_words(vd, d_hi), idesc_pv);
+            else
+              umma_ts_w<1>(tO, tP, desc_words(vd, d_hi), idesc_pv);
+#pragma unroll
+            for (int kk = 1; kk < BN / 16; ++kk)
+              umma_ts_w<1>(tO, tP + kk * 8, desc_words(vd + kk * 128, d_hi), idesc_pv);
+            umma_commit_w(&pv_done[t]);
+            if (j - 1 == n - 1) umma_commit_w(&o_done[t]);
+          }
+          if (WINDOW && ok && !have_k && j < nmax) {
+            ok = warp_all(wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull));
+            have_k = ok;
+          }
+          if (WINDOW && ok && !have_v && j >= 1) {
+            ok = warp_all(wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull));
+            have_v = ok;
+          }
+          if (have_k) umma_commit_w(&kv_empty[Lk % S]);
+          if (have_v) umma_commit_w(&kv_empty[Lv % S]);
         }
-        // A loaded tile that neither query tile uses (a gap between the two
-        // tiles' windows; without a window every loaded tile is used) is still
-        // waited for and released, so the ring keeps its order.
-        if (WINDOW && ok && !have_k && j < nmax) {
-          ok = warp_all(wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull));
-          have_k = ok;
+      } else {
+        for (int j = 0; ok && j <= nmax; ++j) {
+          const uint32_t Lk = L + 2 * j;
+          const uint32_t Lv = L + 2 * j - 1;
+          bool have_k = false, have_v = false;
+#pragma unroll
+          for (int t = 0; t < NQT; ++t) {
+            if (!ok) break;
+            const int n = t ? it.n1 : it.n0;
+            const int s0 = t ? it.s1 : it.s0;  // this tile's first step
+            if (j >= 1 && j - 1 >= s0 && j - 1 < n) {
+              // O_t (+)= P_t(j-1) V_{j-1}. The p_ready arrival for an item's
+              // first step comes after the softmax group read O_t of its
+              // previous item, so O_t is free to be overwritten here.
+              if (!have_v) {
+                if (!(ok = warp_all(wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull))))
+                  break;
+                have_v = true;
+              }
+              if (!(ok = warp_all(wait_bar(&p_ready[t], pw[t] & 1, ctl, kSitePReady)))) break;
+              ++pw[t];
+              tc_fence_after();
+              const uint32_t vd = v_lo + (((Lv % S) * C::kTileBytes) >> 4);
+              const uint32_t tS = tmem + t * BN;
+              const uint32_t tO = tmem + C::kOCol + t * D;
+              // P of keys 16kk..16kk+15: 8 columns. With SPLIT = 1 P fills columns
+              // [64, 128) of S_t; with SPLIT = 2 the two halves of the row sit at
+              // columns [0, 32) and [64, 96), each where its own thread read S.
+              // 16 keys = 16 rows of 128 bytes of V (2048 bytes = 128 in the address field)
+              if (j - 1 == s0)
+                umma_ts_w<0>(tO, tS + p_col<SPLIT>(0), desc_words(vd, d_hi), idesc_pv);
+              else
+                umma_ts_w<1>(tO, tS + p_col<SPLIT>(0), desc_words(vd, d_hi), idesc_pv);
+#pragma unroll
+              for (int kk = 1; kk < BN / 16; ++kk)
+                umma_ts_w<1>(tO, tS + p_col<SPLIT>(kk), desc_words(vd + kk * 128, d_hi), idesc_pv);
+              if (j - 1 == n - 1) umma_commit_w(&o_done[t]);
+            }
+            if (j >= s0 && j < n) {
+              // S_t = Q_t K_j^T
+              if (!have_k) {
+                if (!(ok = warp_all(wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull))))
+                  break;
+                tc_fence_after();
+                have_k = true;
+              }
+              if (j == s0) {
+                if (!(ok = warp_all(wait_bar(&q_full[t], qi[t] & 1, ctl, kSiteQFull)))) break;
+                tc_fence_after();
+              }
+              const uint32_t kd = k_lo + (((Lk % S) * C::kTileBytes) >> 4);
+              const uint32_t qd = q_lo + ((t * C::kTileBytes) >> 4);
+              const uint32_t tS = tmem + t * BN;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+                if (kk == 0)
+                  umma_ss_w<0>(tS, desc_words(qd + koff, d_hi), desc_words(kd + koff, d_hi), idesc_s);
+                else
+                  umma_ss_w<1>(tS, desc_words(qd + koff, d_hi), desc_words(kd + koff, d_hi), idesc_s);
+              }
+              umma_commit_w(&s_ready[t]);
+              if (j == n - 1) umma_commit_w(&q_empty[t]);
+            }
+          }
+          // A loaded tile that neither query tile uses (a gap between the two
+          // tiles' windows; without a window every loaded tile is used) is still
+          // waited for and released, so the ring keeps its order.
+          if (WINDOW && ok && !have_k && j < nmax) {
+            ok = warp_all(wait_bar(&kv_full[Lk % S], (Lk / S) & 1, ctl, kSiteKvFull));
+            have_k = ok;
+          }
+          if (WINDOW && ok && !have_v && j >= 1) {
+            ok = warp_all(wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull));
+            have_v = ok;
+          }
+          if (have_k) umma_commit_w(&kv_empty[Lk % S]);
+          if (have_v) umma_commit_w(&kv_empty[Lv % S]);
         }
-        if (WINDOW && ok && !have_v && j >= 1) {
-          ok = warp_all(wait_bar(&kv_full[Lv % S], (Lv / S) & 1, ctl, kSiteKvFull));
-          have_v = ok;
-        }
-        if (have_k) umma_commit_w(&kv_empty[Lk % S]);
-        if (have_v) umma_commit_w(&kv_empty[Lv % S]);
       }
       L += 2 * nmax;
       qi[0] += it.n0 > it.s0;
@@ -561,9 +674,11 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
     const int hw = (warp >> 2) % SPLIT;
     const int q4 = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * BN + hw * NC;
-    const uint32_t tP = tmem + lane_off + t * BN + p_col<SPLIT>(hw * (NC / 16));
-    const uint32_t tO = tmem + lane_off + C::kOCol + t * D;
+    const uint32_t tS = tmem + lane_off + C::s_col(t) + hw * NC;
+    const uint32_t tP = OWNP ? tmem + lane_off + C::p_base(t)
+                             : tmem + lane_off + t * BN + p_col<SPLIT>(hw * (NC / 16));
+    const uint32_t tO = tmem + lane_off + C::o_col(t);
+    uint32_t np = 0;  // probability tiles written (own-P layout: pv_done phases)
     uint8_t* stg = smem + C::kStgOff + (t * 4 + q4) * C::kStgWarpBytes;  // O staging (hw 0)
     // Split rows: part 1 passes its tile max (then, at the end of an item, its
     // partial row sum) up through xrow; part 0 returns the row max.
@@ -602,6 +717,10 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
           for (int h = 0; h < NC / 32; ++h)
 #pragma unroll
             for (int k = 0; k < 32; ++k) s[h * 32 + k] = __uint_as_float(rr[h][k]);
+        }
+        if (OWNP) {  // S_t read: its columns may take the next scores
+          tc_fence_before();
+          mbar_arrive(&s_free[t]);
         }
         const int kv0 = (it.jb + i) * BN + hw * NC;  // key of s[0]
         const bool edge = (CAUSAL && kv0 + NC - 1 > rt + p.off) || (kv0 + NC > p.Nk);
@@ -657,6 +776,12 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
           if (!(ok = warp_all(wait_bar(&turn[t], tk & 1, ctl, kSiteTurn)))) break;
           ++tk;
         }
+        if (OWNP && np > 0) {
+          // P_t's columns and O_t: the previous P_t V product must be complete.
+          if (!(ok = warp_all(wait_bar(&pv_done[t], (np - 1) & 1, ctl, kSitePvDone)))) break;
+          tc_fence_after();
+        }
+        ++np;
         float lsum;
         if (POLY8 > 0 && !edge && !wedge)
           lsum = exp_tile<T, POLY8, NC>(s, sl2, m_use, tP);
@@ -666,7 +791,8 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
         if (PINGPONG) mbar_arrive(&turn[t ^ 1]);
         if (i > s0 && __any_sync(0xffffffffu, need)) {
           // O_t was last written by PV_t(i-1), complete before S_t(i) was
-          // signalled. Each part of a split row rescales its share of the columns.
+          // signalled (own-P layout: waited for through pv_done above). Each
+          // part of a split row rescales its share of the columns.
 #pragma unroll
           for (int c = hw * (D / 32 / SPLIT); c < (hw + 1) * (D / 32 / SPLIT); ++c) {
             uint32_t o[32];
@@ -723,12 +849,50 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
       }
       const bool has_row = row < p.Nq;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      if constexpr (OUT_F32) {
+        // O in fp32, 32 columns (128 bytes per row) per store: the same
+        // swizzled staging of 32 rows x 128 bytes, one 32 x 32 box per store.
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          if (lane == 0) bulk_wait_group_read0();  // the buffer's previous store has read it
+          __syncwarp();
+          uint32_t o[32];
+          if (n > s0) {
+            tmem_ld_x32(tO + c * 32, o);
+            tmem_wait_ld_x32(o);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float a0, a1;
+            f2_split(f2_mul(f2_make(__uint_as_float(o[e]), __uint_as_float(o[e + 1])),
+                            f2_make(inv_l, inv_l)),
+                     a0, a1);
+            o[e] = __float_as_uint(a0);
+            o[e + 1] = __float_as_uint(a1);
+          }
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            uint4* dst = reinterpret_cast<uint4*>(stg + lane * 128 + ((g ^ (lane & 7)) << 4));
+            *dst = make_uint4(o[4 * g], o[4 * g + 1], o[4 * g + 2], o[4 * g + 3]);
+          }
+          fence_async_smem();
+          __syncwarp();
+          const int y = rt + q4 * 32;
+          if (lane == 0 && y < p.Nq) {
+            tma_store_3d(&tm_o, stg, c * 32, y, it.bh);
+            bulk_commit_group();
+          }
+        }
+      }
       // O in 64-column halves: each lane packs its row's 64 columns into this
       // warp's staging buffer (32 rows x 128 bytes, 128-byte swizzle: 16-byte
       // chunk g of row lane sits at chunk position g ^ (lane % 8)), and one TMA
       // store per half writes the 32 x 64 box (rows past Nq are clipped).
 #pragma unroll
-      for (int half = 0; half < D / 64; ++half) {
+      for (int half = 0; half < (OUT_F32 ? 0 : D / 64); ++half) {
         if (lane == 0) bulk_wait_group_read0();  // the buffer's previous store has read it
         __syncwarp();
 #pragma unroll

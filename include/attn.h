@@ -214,8 +214,36 @@ int attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* ls
 int attn_merge_f16(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                    void* o_out, long long rows, int d, attn_stream_t stream);
 
+/*
+ * Partial results kept in fp32, for a sequence of merges (context-parallel
+ * prefill folds one query block's attention over every key block; rounding
+ * each partial O to bf16 / fp16 before it is merged would add one rounding per
+ * fold). The running-statistics merge is the aikaboom page's "Online Softmax"
+ * applied to whole key blocks.
+ * attn_fwd_partial / attn_fwd_partial_f16: attn_fwd / attn_fwd_f16 (bf16 /
+ *   fp16 q, k, v; same layouts, masks, sizes and errors) except that o is
+ *   float32 [B, Hq, Nq, d] holding O = sum_j softmax_j * v_j unrounded
+ *   (16-byte aligned). No sliding window. Allocates nothing.
+ * attn_merge_partial / attn_merge_partial_f16: attn_merge / attn_merge_f16
+ *   with o_part float32 [rows, d] (such a partial O); o_out, if not NULL,
+ *   receives the merged O rounded to bf16 / fp16.
+ */
+int attn_fwd_partial(const void* q, const void* k, const void* v, float* o, float* lse, int B,
+                     int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                     attn_stream_t stream);
+int attn_fwd_partial_f16(const void* q, const void* k, const void* v, float* o, float* lse, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                         attn_stream_t stream);
+int attn_merge_partial(float* o_acc, float* lse_acc, const float* o_part, const float* lse_part,
+                       void* o_out, long long rows, int d, attn_stream_t stream);
+int attn_merge_partial_f16(float* o_acc, float* lse_acc, const float* o_part,
+                           const float* lse_part, void* o_out, long long rows, int d,
+                           attn_stream_t stream);
+
 /* Number of KV splits attn_decode uses for these sizes on the current device
-   (>= 1; always 1 for d other than 64 and 128), or a negative error code. */
+   (>= 1; always 1 for d other than 64 and 128 and for the persistent pass of
+   d = 128 with 2 to 32 query heads per KV head, which has no fixed split
+   count), or a negative error code. */
 int attn_decode_num_splits(int B, int Hq, int Hkv, int d);
 
 /* The cudaError_t value (as an int) behind the calling thread's most recent

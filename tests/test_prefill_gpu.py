@@ -142,3 +142,39 @@ def test_rejects_bad_arguments_on_gpu(lib):
     with pytest.raises(lib.AttnError) as e:
         lib.attn_fwd(q100, q100, q100)
     assert e.value.code == lib.ATTN_ERR_UNSUPPORTED
+
+
+# The softmax applies a tile's row maximum at the next tile (the running
+# reference moves one tile late, exactly, since O and l keep one reference),
+# and redoes a tile whose maximum exceeds the reference by more than 32 in
+# log2 units. These inputs make the maximum grow at every key tile, or jump.
+MAX_CASES = [
+    # B, Hq, Hkv, N, d, causal, dtype, kind
+    (1, 4, 2, 1000, 128, True, BF16, "ramp"),
+    (1, 4, 2, 1000, 64, True, BF16, "ramp"),
+    (1, 2, 2, 700, 128, False, F16, "ramp"),
+    (1, 4, 2, 1000, 128, True, BF16, "jump"),
+    (1, 4, 4, 900, 64, False, BF16, "jump"),
+    (2, 2, 1, 600, 64, True, F16, "drop"),
+]
+
+
+@pytest.mark.parametrize("case", MAX_CASES, ids=lambda c: "x".join(map(str, c[:5])) + c[7])
+def test_row_maximum_moves(lib, case):
+    B, Hq, Hkv, N, d, causal, dt, kind = case
+    q, k, v = workloads.random_prefill(B, Hq, Hkv, N, N, d, dt, seed=1300 + MAX_CASES.index(case))
+    pos = torch.arange(N, dtype=torch.float32)
+    if kind == "ramp":      # every 128-key tile raises the maxima by well over 8 (log2 units)
+        f = 1.0 + pos / 40.0
+    elif kind == "jump":    # keys from 300 on are 40 times larger: a jump far beyond 32
+        f = torch.where(pos >= 300, 40.0, 1.0)
+    else:                   # large early keys, then small ones: the reference stays high
+        f = torch.where(pos < 200, 12.0, 1.0)
+    k = (k.float() * f[None, None, :, None]).to(dt)
+    # Peaked rows put O close to single value rows; small values keep |O| in
+    # the range where the stated bounds apply (this test is about the maxima).
+    v = (v.float() * 0.25).to(dt)
+    scale = d ** -0.5
+    o, lse = run(lib, q.to(DEV), k.to(DEV), v.to(DEV), scale, causal)
+    o_ref, lse_ref = oracle.attention_ref(q, k, v, scale, causal)
+    compare(o, lse, o_ref, lse_ref, dt, f"moving maximum {case}")
