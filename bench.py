@@ -60,7 +60,8 @@ KERNEL_SOURCES = {
     k: [os.path.join(ROOT, "exact_tiled_attention_38_b200", "csrc", f) for f in files]
     for k, files in {
         "attn_prefill_kernel": ("prefill_sm100.cuh", "common.cuh", "ptx.cuh"),
-        "attn_decode_split_kernel": ("decode_sm100.cuh", "common.cuh", "ptx.cuh"),
+        "attn_decode_persistent_kernel": ("decode_ps_sm100.cuh", "decode_tc_sm100.cuh",
+                                          "decode_sm100.cuh", "common.cuh", "ptx.cuh"),
     }.items()
 }
 
@@ -692,9 +693,9 @@ def run_ours(args, world, rank, local):
         "roofline_decode": {
             "bound": "hbm", "achieved": dec_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": dec_ach / peaks["hbm_gbs"],
-            "traffic": profiled_traffic("attn_decode_split_kernel", DECODE.name),
-            "kernel": "attn_decode_split_kernel<128,4,bf16> + attn_decode_combine_kernel"
-                      " (one attn_decode call, timed together)",
+            "traffic": profiled_traffic("attn_decode_persistent_kernel", DECODE.name),
+            "kernel": "attn_decode_plan_kernel + attn_decode_persistent_kernel<16,4,1,bf16> + "
+                      "attn_decode_gather_kernel (one attn_decode call, timed together)",
             "workload": DECODE.name, "algorithmic_bytes": dbytes, "ms_per_launch": dec_ms,
             "peak_source": f"{src} copy bandwidth (burst)",
             "nominal": {"peak": NOMINAL_PEAKS["hbm_gbs"],
@@ -710,8 +711,8 @@ def run_ours(args, world, rank, local):
                 "segments": e2e_seg, "steps": e2e_steps},
         "clocks": merged_clocks(list(phase_clocks.values())),
         "phases_ms_per_step": phase_ms,
-        # 3 prefill launches + decode split pass + combine per step
-        "gpu_launches": (len(PREFILLS) + 2) * args.steps,
+        # 3 prefill launches + decode plan, stream and gather per step
+        "gpu_launches": (len(PREFILLS) + 3) * args.steps,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()

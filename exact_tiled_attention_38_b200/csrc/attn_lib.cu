@@ -84,6 +84,7 @@ struct PerDeviceOnce {
 
 struct DeviceInfo {
   int sm_count = 0;
+  long long l2_bytes = 0;
   bool sm100 = false;
 };
 
@@ -96,12 +97,14 @@ int device_info(DeviceInfo* out) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ATTN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
   if (!have[dev]) {
-    int major = 0, minor = 0, sms = 0;
+    int major = 0, minor = 0, sms = 0, l2 = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
       return ATTN_ERR_CUDA;
     cache[dev].sm_count = sms;
+    cache[dev].l2_bytes = l2;
     cache[dev].sm100 = (major == 10 && minor == 0);
     have[dev] = true;
   }
@@ -261,6 +264,12 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   return launch_status();
 }
 
+// Prefill knob: KV-head-major order of causal items when K/V exceed L2 (1) or
+// always all heads of a query level together (0).
+#ifndef ETA_PREFILL_HEAD_MAJOR
+#define ETA_PREFILL_HEAD_MAJOR 1
+#endif
+
 // OUT_F32: o is float32 (the unrounded O of a partial result), else T.
 template <typename T, bool OUT_F32 = false>
 int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -335,6 +344,21 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   p.debug_flags = debug_flags;
   p.window = window;
   const int grid = static_cast<int>(total < info.sm_count ? total : info.sm_count);
+  // Causal items go KV head by KV head, in blocks of query levels, when the K
+  // and V of all heads are larger than L2 (otherwise all heads of a query
+  // level run together, which balances the triangular work more finely). A
+  // block holds lcm(grid, group) / group levels: a whole number of rounds.
+  const long long kv_bytes = 2LL * B * Hkv * static_cast<long long>(Nk) * d * 2;
+  p.head_major = 0;
+  if (causal && kv_bytes > info.l2_bytes && ETA_PREFILL_HEAD_MAJOR) {
+    int a = grid, b = p.group;
+    while (b != 0) {
+      const int t = a % b;
+      a = b;
+      b = t;
+    }
+    p.head_major = grid / a;  // lcm(grid, group) / group
+  }
   if constexpr (OUT_F32) {
     if (window > 0) return ATTN_ERR_INVALID;
     if (d == 128)

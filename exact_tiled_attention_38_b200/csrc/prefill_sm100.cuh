@@ -147,6 +147,8 @@ struct Params {
   uint64_t wait_ns;
   int debug_flags;  // bit 0: the producer issues no copies (exercises the wait limit)
   int window;       // causal only: a row keeps its `window` most recent keys (0 = all)
+  int head_major;   // causal: query levels in blocks of this many, KV head by KV head
+                    // inside a block (0: all heads of a level together)
 };
 
 template <typename T>
@@ -259,7 +261,26 @@ template <bool CAUSAL, bool WINDOW = false>
 __device__ __forceinline__ Item decode_item(int idx, const Params& p, int nkv_all) {
   Item it;
   int pair;
-  if (CAUSAL) {  // heaviest (last) query tiles first, all heads of one level together
+  if (CAUSAL && p.head_major > 0) {
+    // K/V of all heads do not fit in L2. Query levels go in blocks of Lb,
+    // heaviest first; inside a block, (batch, KV head) by (batch, KV head),
+    // each taking its Lb levels times the query heads of its group. Lb * group
+    // is a whole number of rounds of the grid, so the CTAs running at one time
+    // stream the K/V of about one KV head, which stays in L2, and every round
+    // has the same weights, which the snake order balances.
+    const int Lb = p.head_major;
+    const int units = p.BH / p.group;  // B * Hkv
+    const int blk = Lb * p.group * units;
+    const int k = idx / blk;
+    const int r = idx - k * blk;
+    const int per_unit = min(Lb, p.n_pairs - k * Lb) * p.group;
+    const int unit = r / per_unit;
+    const int r2 = r - unit * per_unit;
+    const int lvl = k * Lb + r2 / p.group;
+    const int b = unit / p.Hkv;
+    pair = p.n_pairs - 1 - lvl;
+    it.bh = b * p.Hq + (unit - b * p.Hkv) * p.group + (r2 - (r2 / p.group) * p.group);
+  } else if (CAUSAL) {  // heaviest (last) query tiles first, all heads of one level together
     pair = p.n_pairs - 1 - idx / p.BH;
     it.bh = idx - (idx / p.BH) * p.BH;
   } else {  // consecutive items share a head, so concurrent CTAs share K/V in L2
