@@ -60,7 +60,7 @@ KERNEL_SOURCES = {
     k: [os.path.join(ROOT, "exact_tiled_attention_38_b200", "csrc", f) for f in files]
     for k, files in {
         "attn_prefill_kernel": ("prefill_sm100.cuh", "common.cuh", "ptx.cuh"),
-        "attn_decode_persistent_kernel": ("decode_ps_sm100.cuh", "decode_tc_sm100.cuh",
+        "attn_decode_persistent_kernel": ("decode_ps_sm100.cuh",
                                           "decode_sm100.cuh", "common.cuh", "ptx.cuh"),
     }.items()
 }

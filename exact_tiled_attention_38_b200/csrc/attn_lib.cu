@@ -2,12 +2,11 @@
 // encoding, kernel selection, launch configuration and error codes. Every
 // step of the computation runs in the kernels:
 //   prefill_sm100.cuh    prefill, d = 64 / 128 (tcgen05, TMA)
-//   decode_sm100.cuh     decode split pass on CUDA cores (d = 64, groups <= 4)
-//                        and the LSE combine
+//   decode_sm100.cuh     decode split pass on CUDA cores (d = 64; d = 128
+//                        with one query head per KV head), the LSE combine
+//                        and the token-offset scan of large batches
 //   decode_ps_sm100.cuh  decode as one persistent streaming pass on tcgen05
 //                        (d = 128, groups 2..32): plan, stream, gather
-//   decode_tc_sm100.cuh  helpers of the tcgen05 decode (and its earlier
-//                        one-CTA-per-split pass, kept as a knob)
 //   generic_fwd.cuh      prefill and decode for the other head sizes
 //   merge.cuh            LSE merge of partial results (context parallelism)
 #include <cuda.h>
@@ -22,7 +21,6 @@
 #include "../../include/attn.h"
 #include "decode_ps_sm100.cuh"
 #include "decode_sm100.cuh"
-#include "decode_tc_sm100.cuh"
 #include "generic_fwd.cuh"
 #include "merge.cuh"
 #include "prefill_sm100.cuh"
@@ -312,6 +310,7 @@ int fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     g.window = window;
     g.scale_log2 = scale * 1.4426950408889634f;
     g.seqlens = nullptr;
+    g.tok_off = nullptr;
     return launch_generic<T, OUT_F32>(g, B * Hq, Nq, st);
   }
 
@@ -396,27 +395,15 @@ inline int decode_group_tile(int G) { return (G <= 4 || ETA_DECODE_MAX_GP == 4) 
 #ifndef ETA_DECODE_WAVES
 #define ETA_DECODE_WAVES 8
 #endif
-// Tensor-core split pass (d = 128): used for groups of ETA_DECODE_TC_MIN_G to
-// 32 query heads per KV head, where the CUDA-core pass is bound by its fp32
-// reductions rather than by HBM. One CTA per SM (its ring holds 3 x 64 KB),
-// about ETA_DECODE_TC_WAVES waves of split CTAs.
-#ifndef ETA_DECODE_TC_MIN_G
-#define ETA_DECODE_TC_MIN_G 8
-#endif
-// Two waves measured best on B200 (B = 64, 1K-8K tokens): 0.250 / 0.146 /
-// 0.095 ms for groups of 8 / 16 / 32 against 0.260 / 0.162 / 0.136 ms with 8
-// waves; more CTAs only add their fixed costs.
-#ifndef ETA_DECODE_TC_WAVES
-#define ETA_DECODE_TC_WAVES 2
-#endif
 // Persistent streaming pass (decode_ps_sm100.cuh) for d = 128 and
 // ETA_DECODE_PS_MIN_G to 32 query heads per KV head; 0 turns it off (the
-// one-CTA-per-split tensor-core pass then takes groups of 8 to 32). Measured
-// on B200 (64 sequences of 1K-8K tokens, d = 128, median of 30 launches, L2
-// flushed): group 4 0.236 ms against 0.246 ms on the CUDA-core pass, group 8
-// 0.238 / 0.248 ms and group 16 0.240 / 0.256 ms against the one-CTA-per-split
-// tensor-core pass, MQA 0.088 / 0.099 ms; a single head per KV head (MHA)
-// 0.236 ms against 0.232 ms on the CUDA-core pass, which keeps it.
+// CUDA-core split pass then takes every group). Measured on B200 (64
+// sequences of 1K-8K tokens, d = 128, median of 30 launches, L2 flushed):
+// group 4 0.236 ms against 0.246 ms on the CUDA-core pass; groups of 8 / 16 /
+// 32 0.238 / 0.240 / 0.088 ms against 0.248 / 0.256 / 0.099 ms on an earlier
+// tensor-core pass with one CTA per (sequence, KV head, split) and a combine
+// kernel (removed); a single head per KV head (MHA) 0.236 ms against 0.232 ms
+// on the CUDA-core pass, which keeps it.
 #ifndef ETA_DECODE_PS_MIN_G
 #define ETA_DECODE_PS_MIN_G 2
 #endif
@@ -427,9 +414,6 @@ inline int decode_group_tile(int G) { return (G <= 4 || ETA_DECODE_MAX_GP == 4) 
 #endif
 inline bool decode_use_ps(int G, int d) {
   return ETA_DECODE_PS_MIN_G > 0 && d == 128 && G >= ETA_DECODE_PS_MIN_G && G <= 32;
-}
-inline bool decode_use_tc(int G, int d) {
-  return !decode_use_ps(G, d) && d == 128 && G >= ETA_DECODE_TC_MIN_G && G <= 32;
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -460,15 +444,8 @@ inline PsLayout ps_layout(int B, int Hkv, int G, int nc, bool partials) {
   return L;
 }
 
-int decode_splits(int B, int Hq, int Hkv, int d, int sm_count) {
+int decode_splits(int B, int Hq, int Hkv, int sm_count) {
   const int G = Hq / Hkv;
-  if (decode_use_tc(G, d)) {
-    const long long units = static_cast<long long>(B) * Hkv;
-    long long ns = units > 0 ? (ETA_DECODE_TC_WAVES * static_cast<long long>(sm_count) + units - 1) / units : 1;
-    if (ns < 1) ns = 1;
-    if (ns > 64) ns = 64;
-    return static_cast<int>(ns);
-  }
   const int GP = decode_group_tile(G);
   const int nchunk = (G + GP - 1) / GP;
   const long long units = static_cast<long long>(B) * Hkv * nchunk;
@@ -494,18 +471,15 @@ int launch_decode_split(const decode::DParams& p, cudaStream_t st) {
   return launch_status();
 }
 
-template <int NP, typename T>
-int launch_decode_tc(const decode::DParams& p, cudaStream_t st) {
-  auto kern = decode_tc::attn_decode_tc_kernel<NP, T>;
-  constexpr int smem = decode_tc::TCfg<NP>::kSmemBytes;
-  static PerDeviceOnce attr;
-  const cudaError_t attr_err = attr.run([&]() {
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err);
-  const dim3 grid(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(p.Hkv),
-                  static_cast<unsigned>(p.B));
-  kern<<<grid, decode_tc::kThreads, smem, st>>>(p);
+// Token offsets of a large batch's sequences in the packed cache (one scan
+// per call); smaller batches leave `tok_off` NULL and each CTA sums at most
+// kOffsetsMinBatch lengths itself.
+inline bool decode_needs_offsets(int B) { return B > decode::kOffsetsMinBatch; }
+inline size_t offsets_bytes(int B) {
+  return decode_needs_offsets(B) ? align_up(static_cast<size_t>(B) * 8, 256) : 0;
+}
+int launch_decode_offsets(const int32_t* seqlens, long long* tok_off, int B, cudaStream_t st) {
+  decode::attn_decode_offsets_kernel<<<1, decode::kOffThreads, 0, st>>>(seqlens, tok_off, B);
   return launch_status();
 }
 
@@ -602,10 +576,9 @@ int launch_decode_combine(const float* po, const float* pl, void* o, float* lse,
 
 template <int D, typename T>
 int decode_launch_all(const decode::DParams& p, void* o, float* lse, cudaStream_t st) {
-  if (decode_use_tc(p.G, D)) {
-    const int rc = p.G <= 16 ? launch_decode_tc<16, T>(p, st) : launch_decode_tc<32, T>(p, st);
-    if (rc != ATTN_OK || p.o != nullptr) return rc;  // one split writes o and lse itself
-    return launch_decode_combine<D, T>(p.part_o, p.part_lse, o, lse, p.B * p.Hq, p.nsplit, st);
+  if (p.tok_off != nullptr) {
+    const int rc = launch_decode_offsets(p.seqlens, const_cast<long long*>(p.tok_off), p.B, st);
+    if (rc != ATTN_OK) return rc;
   }
 #if ETA_DECODE_MAX_GP == 8
   const int GP = decode_group_tile(p.G);
@@ -618,11 +591,16 @@ int decode_launch_all(const decode::DParams& p, void* o, float* lse, cudaStream_
 }
 
 // Decode for head sizes other than 64 and 128: the generic kernel in decode
-// mode, one CTA per (sequence, query head), no workspace.
+// mode, one CTA per (sequence, query head). `tok_off`: room for B token
+// offsets, filled here by the scan, or NULL (each CTA sums them).
 template <typename T>
 int decode_generic(const void* q, const void* kc, const void* vc, const int32_t* seqlens,
                    void* o, float* lse, int B, int Hq, int Hkv, int d, float scale, int window,
-                   cudaStream_t st) {
+                   long long* tok_off, cudaStream_t st) {
+  if (tok_off != nullptr) {
+    const int rc = launch_decode_offsets(seqlens, tok_off, B, st);
+    if (rc != ATTN_OK) return rc;
+  }
   generic::GParams g;
   g.q = q;
   g.k = kc;
@@ -640,6 +618,7 @@ int decode_generic(const void* q, const void* kc, const void* vc, const int32_t*
   g.window = window;
   g.scale_log2 = scale * 1.4426950408889634f;
   g.seqlens = seqlens;
+  g.tok_off = tok_off;
   return launch_generic<T>(g, B * Hq, 1, st);
 }
 
@@ -660,13 +639,25 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
   DeviceInfo info;
   if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
   if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
-  if (!tensor_core_d(d))
-    return decode_generic<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, window, st);
+  cudaMemPool_t pool;
+  if (!tensor_core_d(d)) {
+    if (!decode_needs_offsets(B))
+      return decode_generic<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, window,
+                               nullptr, st);
+    void* ws = nullptr;
+    if (workspace_pool(&pool) != ATTN_OK) return ATTN_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(&ws, offsets_bytes(B), pool, st) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    const int rc = decode_generic<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, window,
+                                     static_cast<long long*>(ws), st);
+    const cudaError_t fe = cudaFreeAsync(ws, st);
+    if (rc != ATTN_OK) return rc;
+    return fe == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
   if (decode_use_ps(Hq / Hkv, d)) {
     const int nc = info.sm_count;
     const PsLayout L = ps_layout(B, Hkv, Hq / Hkv, nc, true);
     void* ws = nullptr;
-    cudaMemPool_t pool;
     if (workspace_pool(&pool) != ATTN_OK) return ATTN_ERR_CUDA;
     if (cudaMallocFromPoolAsync(&ws, L.total, pool, st) != cudaSuccess) return ATTN_ERR_CUDA;
     const int rc = decode_ps_run<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, scale, window,
@@ -687,29 +678,20 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
   p.G = Hq / Hkv;
   const int GP = decode_group_tile(p.G);
   p.nchunk = (p.G + GP - 1) / GP;
-  p.nsplit = decode_splits(B, Hq, Hkv, d, info.sm_count);
+  p.nsplit = decode_splits(B, Hq, Hkv, info.sm_count);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
   p.window = window;
-  p.o = nullptr;
-  p.lse = nullptr;
-  if (decode_use_tc(p.G, d) && p.nsplit == 1) {
-    // One split per sequence: the tensor-core pass writes the result; no
-    // workspace, no combine.
-    p.o = o;
-    p.lse = lse;
-    p.part_o = nullptr;
-    p.part_lse = nullptr;
-    return decode_launch_all<128, T>(p, o, lse, st);
-  }
 
+  // Workspace: the token offsets (large batches), then the split partials.
   const size_t rows = static_cast<size_t>(B) * Hq;
-  const size_t bytes = static_cast<size_t>(p.nsplit) * rows * (d + 1) * sizeof(float);
+  const size_t off_bytes = offsets_bytes(B);
+  const size_t bytes = off_bytes + static_cast<size_t>(p.nsplit) * rows * (d + 1) * sizeof(float);
   void* ws = nullptr;
-  cudaMemPool_t pool;
   if (workspace_pool(&pool) != ATTN_OK) return ATTN_ERR_CUDA;
   if (cudaMallocFromPoolAsync(&ws, bytes, pool, st) != cudaSuccess) return ATTN_ERR_CUDA;
-  p.part_o = reinterpret_cast<float*>(ws);
+  p.tok_off = off_bytes ? static_cast<long long*>(ws) : nullptr;
+  p.part_o = reinterpret_cast<float*>(static_cast<char*>(ws) + off_bytes);
   p.part_lse = p.part_o + static_cast<size_t>(p.nsplit) * rows * d;
   const int rc = d == 128 ? decode_launch_all<128, T>(p, o, lse, st)
                           : decode_launch_all<64, T>(p, o, lse, st);
@@ -788,7 +770,7 @@ int attn_decode_num_splits(int B, int Hq, int Hkv, int d) {
   if (eta::api::decode_use_ps(Hq / Hkv, d)) return 1;  // one streaming pass, no fixed split
   eta::api::DeviceInfo info;
   if (eta::api::device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
-  return eta::api::decode_splits(B, Hq, Hkv, d, info.sm_count);
+  return eta::api::decode_splits(B, Hq, Hkv, info.sm_count);
 }
 
 const char* attn_strerror(int code) {
@@ -1000,11 +982,20 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
       !aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(o, 16) ||
       !aligned(seqlens, 4) || (lse != nullptr && !aligned(lse, 4)))
     return ATTN_ERR_INVALID;
-  if (!tensor_core_d(d)) {  // the generic kernel needs no scratch
+  if (!tensor_core_d(d)) {
+    // The generic kernel needs scratch only for the token offsets of a large
+    // batch; beyond the scratch's capacity (a million sequences) each CTA
+    // sums them itself.
     DeviceInfo info;
     if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
     if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
-    return decode_generic<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, 0, st);
+    long long* tok_off = nullptr;
+    if (decode_needs_offsets(B) && offsets_bytes(B) <= kNoAllocScratchFloats * sizeof(float)) {
+      float* scratch = nullptr;
+      if (noalloc_scratch(&scratch) != ATTN_OK) return ATTN_ERR_CUDA;
+      tok_off = reinterpret_cast<long long*>(scratch);
+    }
+    return decode_generic<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, 0, tok_off, st);
   }
   DeviceInfo info;
   if (device_info(&info) != ATTN_OK) return ATTN_ERR_CUDA;
@@ -1034,39 +1025,29 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
   p.G = Hq / Hkv;
   const int GP = decode_group_tile(p.G);
   p.nchunk = (p.G + GP - 1) / GP;
-  // One split needs B * Hq * (d + 1) floats of scratch; fewer splits than
-  // attn_decode's count are used when that count does not fit. The
-  // tensor-core pass with a single split writes o and lse itself and needs no
-  // scratch, so it runs even when not one split fits; every other case where
-  // not one split fits is refused.
+  // Scratch: the token offsets of a large batch, then the split partials.
+  // One split needs B * Hq * (d + 1) floats; fewer splits than attn_decode's
+  // count are used when that count does not fit, and a call where not one
+  // split fits is refused.
   const size_t rows = static_cast<size_t>(B) * Hq;
-  const size_t per_split = rows * (d + 1);
-  const size_t fit = kNoAllocScratchFloats / per_split;
-  const int want = decode_splits(B, Hq, Hkv, d, info.sm_count);
-  const bool tc = decode_use_tc(p.G, d);
+  const size_t off_bytes = offsets_bytes(B);
+  const size_t cap = kNoAllocScratchFloats * sizeof(float);
+  const size_t per_split = rows * (d + 1) * sizeof(float);
+  const size_t fit = off_bytes < cap ? (cap - off_bytes) / per_split : 0;
+  const int want = decode_splits(B, Hq, Hkv, info.sm_count);
   p.nsplit = static_cast<int>(fit < static_cast<size_t>(want) ? fit : want);
-  if (p.nsplit < 1) {
-    if (!tc) return ATTN_ERR_SCRATCH;
-    p.nsplit = 1;
-  }
+  if (p.nsplit < 1) return ATTN_ERR_SCRATCH;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
   p.window = 0;
-  p.o = nullptr;
-  p.lse = nullptr;
-  if (tc && p.nsplit == 1) {  // writes the result directly; no scratch
-    p.o = o;
-    p.lse = lse;
-    p.part_o = nullptr;
-    p.part_lse = nullptr;
-    return decode_launch_all<128, T>(p, o, lse, st);
-  }
   float* scratch = nullptr;
   if (noalloc_scratch(&scratch) != ATTN_OK) return ATTN_ERR_CUDA;
-  // Every partial slot is written by the split pass before the combine reads
-  // it, so nothing in the scratch has to start at zero.
-  p.part_o = scratch;
-  p.part_lse = scratch + static_cast<size_t>(p.nsplit) * rows * d;
+  // Every offset and partial slot is written before it is read, so nothing
+  // in the scratch has to start at zero.
+  char* base = reinterpret_cast<char*>(scratch);
+  p.tok_off = off_bytes ? reinterpret_cast<long long*>(base) : nullptr;
+  p.part_o = reinterpret_cast<float*>(base + off_bytes);
+  p.part_lse = p.part_o + static_cast<size_t>(p.nsplit) * rows * d;
   return d == 128 ? decode_launch_all<128, T>(p, o, lse, st)
                   : decode_launch_all<64, T>(p, o, lse, st);
 }

@@ -54,7 +54,7 @@
 #include <type_traits>
 
 #include "common.cuh"
-#include "decode_tc_sm100.cuh"
+#include "decode_sm100.cuh"
 
 namespace eta {
 namespace decode_ps {
@@ -90,6 +90,48 @@ enum : unsigned {
   kSiteDrain = 0x48,
   kSiteQFree = 0x49,
 };
+
+// Byte offset of 16-byte unit u (0..15 along a 256-byte row) of row r in a
+// tile of two 128-byte-swizzled boxes (columns 0-63 | 64-127), box_bytes apart.
+__device__ __forceinline__ uint32_t sw128_off(int r, int u, int box_bytes) {
+  return static_cast<uint32_t>((u >> 3) * box_bytes + r * 128 + (((u & 7) ^ (r & 7)) << 4));
+}
+
+// Tensor-memory loads and stores of NP (16 or 32) consecutive columns.
+template <int NP>
+__device__ __forceinline__ void tmem_ld_np(uint32_t taddr, uint32_t (&r)[NP]);
+template <>
+__device__ __forceinline__ void tmem_ld_np<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  tmem_ld_x16(taddr, r);
+  tmem_wait_ld_x16(r);
+}
+template <>
+__device__ __forceinline__ void tmem_ld_np<32>(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_ld_x32(taddr, r);
+  tmem_wait_ld_x32(r);
+}
+template <int NP>
+__device__ __forceinline__ void tmem_st_np(uint32_t taddr, const uint32_t (&r)[NP]);
+template <>
+__device__ __forceinline__ void tmem_st_np<16>(uint32_t taddr, const uint32_t (&r)[16]) {
+  tmem_st_x16(taddr, r);
+}
+template <>
+__device__ __forceinline__ void tmem_st_np<32>(uint32_t taddr, const uint32_t (&r)[32]) {
+  tmem_st_x32(taddr, r);
+}
+
+// fp32 -> bf16 / fp16 bits, round to nearest even.
+template <typename T>
+__device__ __forceinline__ uint16_t to_bits(float x);
+template <>
+__device__ __forceinline__ uint16_t to_bits<__nv_bfloat16>(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+template <>
+__device__ __forceinline__ uint16_t to_bits<__half>(float x) {
+  return __half_as_ushort(__float2half_rn(x));
+}
 
 struct PParams {
   const void* q;
@@ -374,10 +416,6 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
   using C = PCfg<NP>;
   using R = Roles<HS>;
   constexpr int GPT = GP / HS;  // heads per softmax thread
-  using decode_tc::sw128_off;
-  using decode_tc::tmem_ld_np;
-  using decode_tc::tmem_st_np;
-  using decode_tc::to_bits;
   const int c = blockIdx.x;
 
   extern __shared__ uint8_t smem_raw[];

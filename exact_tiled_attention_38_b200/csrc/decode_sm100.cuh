@@ -22,8 +22,11 @@
 //
 // Packed cache layout: sequence b starts at token offset sum_{j<b} L_j and is
 // stored [Hkv][L_b][d], so one (sequence, KV head) is one contiguous run. The
-// offsets are recomputed on the device from `seqlens`; negative lengths count
-// as 0; an empty sequence gives O = 0 and LSE = -inf.
+// offsets come from `seqlens` on the device: for batches above 1024 sequences
+// from one prefix sum per call (attn_decode_offsets_kernel below; the
+// persistent pass has its own in its plan kernel), else summed by each CTA
+// over at most 1024 lengths; negative lengths count as 0; an empty sequence
+// gives O = 0 and LSE = -inf.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -78,10 +81,9 @@ struct DParams {
   const void* kc;
   const void* vc;
   const int* seqlens;
+  const long long* tok_off;  // [B] token offsets of the sequences, or NULL: summed per CTA
   float* part_o;    // [nsplit][B][Hq][D]
   float* part_lse;  // [nsplit][B][Hq], log2 units
-  void* o;          // tensor-core split pass with nsplit == 1: the output itself, else NULL
-  float* lse;       //   and its LSE (natural log, may be NULL)
   int B;
   int Hq;
   int Hkv;
@@ -151,12 +153,15 @@ __global__ void __launch_bounds__(kThreads) attn_decode_split_kernel(const DPara
   const int b = blockIdx.z;
 
   if (warp == 0) {
+    // The sequence's token offset: computed once for the call by the offsets
+    // kernel when the batch is large, else summed here (B <= 1024 lengths).
     long long acc = 0;
-    for (int j = lane; j < b; j += 32) acc += max(p.seqlens[j], 0);
+    if (p.tok_off == nullptr)
+      for (int j = lane; j < b; j += 32) acc += max(p.seqlens[j], 0);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) {
-      misc[0] = acc;
+      misc[0] = p.tok_off != nullptr ? p.tok_off[b] : acc;
       misc[1] = max(p.seqlens[b], 0);
     }
   }
@@ -384,6 +389,45 @@ __global__ void __launch_bounds__(kThreads) attn_decode_split_kernel(const DPara
     const size_t row = (static_cast<size_t>(split) * p.B + b) * p.Hq + hq;
     p.part_o[row * D + dim] = Lsum > 0.f ? acc / Lsum : 0.f;
     if (dim == 0) p.part_lse[row] = Lsum > 0.f ? M + lg2_approx(Lsum) : -INFINITY;
+  }
+}
+
+// Token offsets of the packed cache for large batches: tok_off[b] = the sum
+// of max(L_j, 0) over j < b, as an exclusive prefix sum in one CTA, 1024
+// consecutive sequences per round (coalesced reads of seqlens, a warp scan,
+// then a scan of the warp totals; the running total carries over rounds).
+constexpr int kOffThreads = 1024;
+constexpr int kOffsetsMinBatch = 1024;  // smaller batches sum their offsets per CTA
+
+__global__ void __launch_bounds__(kOffThreads) attn_decode_offsets_kernel(
+    const int* __restrict__ seqlens, long long* __restrict__ tok_off, int B) {
+  __shared__ long long s_w[kOffThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long carry = 0;
+  for (int base = 0; base < B; base += kOffThreads) {
+    const int b = base + static_cast<int>(threadIdx.x);
+    const long long len = b < B ? max(seqlens[b], 0) : 0;
+    long long x = len;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_w[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      long long w = s_w[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      s_w[lane] = w;
+    }
+    __syncthreads();
+    if (b < B) tok_off[b] = carry + x - len + (warp > 0 ? s_w[warp - 1] : 0);
+    carry += s_w[31];
+    __syncthreads();  // s_w is rewritten in the next round
   }
 }
 

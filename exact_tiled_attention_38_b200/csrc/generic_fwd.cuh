@@ -10,8 +10,9 @@
 //
 // Decode mode (seqlens != NULL): one query row per (batch, query head) over the
 // packed ragged cache of attn_decode (sequence b at token offset
-// sum_{j<b} L_j, laid out [Hkv][L_b][d]); it is the causal case with Nq = 1
-// and Nk = L_b, so a window keeps the last W cached tokens.
+// sum_{j<b} L_j, laid out [Hkv][L_b][d]; the offsets from one prefix sum per
+// call when given, else summed per CTA); it is the causal case with Nq = 1 and
+// Nk = L_b, so a window keeps the last W cached tokens.
 //
 // Layout of the work: a CTA of 4 warps owns 16 query rows of one (batch, query
 // head), 4 rows per warp. Per 32-key tile the whole CTA stages K and V in
@@ -56,6 +57,7 @@ struct GParams {
   int window;  // causal only; 0 = no window
   float scale_log2;
   const int* seqlens;  // decode mode when not NULL (Nq = 1, Nk = L_b, causal)
+  const long long* tok_off;  // decode: [B] token offsets, or NULL: summed per CTA
 };
 
 // Shared-memory row stride in bytes for d 16-bit elements (+16 bytes of pad).
@@ -148,11 +150,12 @@ __global__ void __launch_bounds__(kThreads) attn_generic_kernel(const GParams p)
     __shared__ int s_len;
     if (warp == 0) {
       long long acc = 0;
-      for (int j = lane; j < b; j += 32) acc += max(p.seqlens[j], 0);
+      if (p.tok_off == nullptr)
+        for (int j = lane; j < b; j += 32) acc += max(p.seqlens[j], 0);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) {
-        s_tok = acc;
+        s_tok = p.tok_off != nullptr ? p.tok_off[b] : acc;
         s_len = max(p.seqlens[b], 0);
       }
     }

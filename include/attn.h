@@ -106,17 +106,21 @@ int attn_fwd_f16(const void* q, const void* k, const void* v, void* o, float* ls
  * Sizes: B >= 0 (0: nothing to do), Hq >= 1, Hkv >= 1, Hq % Hkv == 0,
  * d a multiple of 8 in [8, 256], B * Hq < 2^29; for d = 64 and 128 also
  * B <= 65,535 (larger B returns ATTN_ERR_UNSUPPORTED).
- * For d = 64 and 128, allocates a split-KV scratch of nsplit * B * Hq * (d + 1) * 4 bytes with
- * cudaMallocFromPoolAsync on `stream` and frees it with cudaFreeAsync on the
- * same stream (stream-ordered; no block outlives the call's work). The pool is
- * the library's own, one per device, created on first use; it keeps up to
- * 256 MiB of freed blocks cached, so callers that synchronise between calls do
- * not pay for re-mapping device memory each time. The caller's pools are not
- * touched. Other d use one block per (sequence, query head), no split and no
- * scratch. With d = 128 and 8 to 32 query heads per KV head the split pass runs
- * on the tensor cores; when it uses one split per sequence
- * (attn_decode_num_splits returns 1) it writes o and lse itself and nothing is
- * allocated.
+ * Device memory: the call takes one workspace block from cudaMallocFromPoolAsync
+ * on `stream` and returns it with cudaFreeAsync on the same stream
+ * (stream-ordered; no block outlives the call's work). Its size:
+ *   - d = 128 with 2 to 32 query heads per KV head (G = Hq / Hkv), the
+ *     persistent tensor-core pass: B * 8 + (B + 1) * 4 bytes of per-sequence
+ *     offsets, 16 bytes per SM, and (B * Hkv + SMs - 1) * G * (d + 1) * 4 bytes
+ *     of partial results, each part rounded up to 256 bytes;
+ *   - other d = 64 and 128 cases, the CUDA-core split pass: nsplit * B * Hq *
+ *     (d + 1) * 4 bytes of split partials (nsplit = attn_decode_num_splits),
+ *     plus B * 8 bytes of token offsets when B > 1024;
+ *   - other d: B * 8 bytes of token offsets when B > 1024, else nothing.
+ * The pool is the library's own, one per device, created on first use; it
+ * keeps up to 256 MiB of freed blocks cached, so callers that synchronise
+ * between calls do not pay for re-mapping device memory each time. The
+ * caller's pools are not touched.
  */
 int attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
                 void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
@@ -134,17 +138,23 @@ int attn_decode_f16(const void* q, const void* kcache, const void* vcache,
  * pool at start-up, a latency-critical path where an allocator call may lock
  * or synchronise, or a runtime whose memory plan is fixed before serving.
  * Same arguments, layout and results as attn_decode (bf16), except:
- *   - The split-KV scratch is a fixed array of 2,097,152 floats (8 MiB) in
- *     this library's device memory, held by every GPU that loads the library
+ *   - The workspace is a fixed array of 2,097,152 floats (8 MiB) in this
+ *     library's device memory, held by every GPU that loads the library
  *     until the process exits. It calls no cudaMalloc/cudaFree and no
  *     allocating library routine.
- *   - One split needs B * Hq * (d + 1) floats. When the usual split count does
- *     not fit, fewer splits are used (results then agree with attn_decode to
- *     rounding). When not even one split fits: with d = 128 and 8 to 32 query
- *     heads per KV head the tensor-core pass runs with one split and writes o
- *     and lse itself, using no scratch; any other such call returns
- *     ATTN_ERR_SCRATCH and enqueues nothing. Head sizes other than 64 and 128
- *     never use the scratch.
+ *   - Persistent tensor-core pass (d = 128, 2 to 32 query heads per KV head):
+ *     when its partial results (sizes as in attn_decode) do not fit, each SM
+ *     takes whole (sequence, KV head) segments and writes o and lse itself;
+ *     only the per-sequence offsets (under 1 MB for B <= 65,535) are kept in
+ *     the array, so these calls are never refused. Results agree with
+ *     attn_decode to rounding.
+ *   - CUDA-core split pass (other d = 64 and 128 cases): one split needs
+ *     B * Hq * (d + 1) floats besides the token offsets of a batch above 1024
+ *     sequences. When the usual split count does not fit, fewer splits are
+ *     used (results then agree with attn_decode to rounding); when not one
+ *     split fits the call returns ATTN_ERR_SCRATCH and enqueues nothing.
+ *   - Other d keep only the token offsets of a batch above 1024 sequences in
+ *     the array (beyond a million sequences each block sums them itself).
  *   - The first call on a device looks up the array's device address (a
  *     runtime call); make that first call before any stream capture. The
  *     address is remembered with the id of the device's context; after

@@ -4,9 +4,11 @@ Covers the ragged GQA workload at full size (64 sequences, lengths uniform in
 [1024, 8192]) and small cases: length 1, empty sequences, lengths that are not
 multiples of the 32-key stage, MQA (one KV head for 32 query heads), MHA, a
 group of 3 (padded to 4), group 8, d = 64 and fp16, a single long sequence
-spread over many splits; and, for the tensor-core split pass (groups of 8 to
+spread over many splits; for the persistent tensor-core pass (groups of 2 to
 32 with d = 128), tile tails, padded groups, MQA, the workload's scale with
-groups of 8, and keys that move the running maximum at every tile.
+groups of 8, keys that move the running maximum at every tile, and segments
+cut between CTAs; and batches of twenty thousand short sequences, whose token
+offsets come from one prefix sum per call, on every decode path.
 """
 import numpy as np
 import pytest
@@ -102,8 +104,9 @@ def test_decode_rejects_bad_arguments(lib):
     assert e.value.code == lib.ATTN_ERR_INVALID
 
 
-# Groups of 8 to 32 query heads per KV head with d = 128 take the tensor-core
-# split pass (scores and P V as tcgen05 products, keys on tensor-memory lanes).
+# Groups of 2 to 32 query heads per KV head with d = 128 take the persistent
+# tensor-core pass (scores and P V as tcgen05 products, keys on tensor-memory
+# lanes).
 TC_CASES = [
     # B, Hq, Hkv, d, lengths, dtype
     (4, 16, 2, 128, [1, 127, 128, 129], BF16),         # tile tails around 128 keys
@@ -149,9 +152,9 @@ def test_decode_tensor_core_running_max_moves(lib):
 
 
 def test_decode_tensor_core_single_split_writes_output(lib):
-    # B * Hkv >= 2 waves of CTAs: one split per sequence, so the tensor-core
-    # pass writes O and LSE itself (no workspace, no combine). Includes empty
-    # and very short sequences, fp16, and the call without LSE.
+    # Many short segments: most are whole in one CTA, whose epilogue writes O
+    # and LSE itself (no partials). Includes empty and very short sequences,
+    # fp16, and the call without LSE.
     B, Hq, Hkv, d = 40, 64, 8, 128
     sl = workloads.decode_seqlens(B, 0, 300, 2400)
     sl[3] = 0
@@ -197,3 +200,32 @@ def test_decode_persistent_cuts(lib, case):
     assert torch.equal(o, o2) and torch.equal(lse, lse2)  # fixed assignment: bitwise repeatable
     o_ref, lse_ref = oracle.decode_ref(q, kc, vc, sl, scale, Hkv)
     compare(o, lse, o_ref, lse_ref, dt, f"persistent {case[:3]}")
+
+
+# Batches above 1024 sequences: each sequence's offset in the packed cache
+# comes from one prefix-sum kernel per call (the plan kernel on the persistent
+# pass) instead of each CTA summing the lengths before its own.
+BIG_B_CASES = [
+    # B, Hq, Hkv, d, dtype; lengths uniform in [0, 48], every 11th empty
+    (20000, 4, 4, 128, BF16),   # MHA: CUDA-core split pass
+    (20000, 8, 2, 64, F16),     # d = 64, group 4: CUDA-core split pass
+    (20000, 4, 2, 96, BF16),    # d = 96: generic kernel
+    (20000, 16, 2, 128, BF16),  # group 8: persistent pass
+]
+
+
+def big_batch(case, seed):
+    B, Hq, Hkv, d, dt = case
+    sl = workloads.decode_seqlens(B, 0, 48, seed)
+    sl[::11] = 0
+    return workloads.random_decode(B, Hq, Hkv, d, sl, dt, seed=seed + 1)
+
+
+@pytest.mark.parametrize("case", BIG_B_CASES, ids=lambda c: f"B{c[0]}h{c[1]}kv{c[2]}d{c[3]}")
+def test_decode_large_batch_offsets(lib, case):
+    B, Hq, Hkv, d, dt = case
+    q, kc, vc, sl = big_batch(case, 2700 + BIG_B_CASES.index(case))
+    scale = d ** -0.5
+    o, lse = run(lib, q.to(DEV), kc.to(DEV), vc.to(DEV), sl.to(DEV), Hkv, scale)
+    o_ref, lse_ref = oracle.decode_ref(q, kc, vc, sl, scale, Hkv)
+    compare(o, lse, o_ref, lse_ref, dt, f"large batch {case[:4]}")

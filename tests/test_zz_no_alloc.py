@@ -121,11 +121,30 @@ def test_noalloc_refuses_sizes_beyond_its_scratch(lib):
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,lens", [
-    (3, 32, 4, [2000, 10, 700]),   # tensor-core split pass, several splits in the scratch
-    (40, 64, 8, None),             # tensor-core pass, one split: writes o and lse itself
+    (3, 32, 4, [2000, 10, 700]),   # persistent pass, one segment cut over many CTAs
+    (40, 64, 8, None),             # persistent pass, short segments mostly whole in one CTA
 ])
 def test_noalloc_tensor_core_groups(lib, B, Hq, Hkv, lens):
     sl = torch.tensor(lens, dtype=torch.int32) if lens else workloads.decode_seqlens(B, 0, 400, 41)
     q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, 128, sl, torch.bfloat16, seed=43,
                                             device=DEV)
     _call_pair(lib, q, kc, vc, sl, Hkv)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d", [
+    (3000, 1, 1, 128),    # CUDA-core split pass: offsets, then a few splits in the scratch
+    (20000, 4, 2, 96),    # generic kernel: only the offsets in the scratch
+    (20000, 16, 2, 128),  # persistent pass: plan only, whole segments per CTA
+])
+def test_noalloc_large_batch_offsets(lib, B, Hq, Hkv, d):
+    # Above 1024 sequences the token offsets come from one prefix sum per call,
+    # kept in the scratch ahead of whatever else the pass needs there.
+    sl = workloads.decode_seqlens(B, 0, 48, 57)
+    sl[::11] = 0
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, d, sl, torch.bfloat16, seed=59,
+                                            device=DEV)
+    _call_pair(lib, q, kc, vc, sl, Hkv)
+    o, lse = lib.attn_decode_noalloc(q, kc, vc, sl, Hkv=Hkv)
+    torch.cuda.synchronize()
+    _oracle_sample(q, kc, vc, sl, Hkv, o, lse, list(range(0, B, 97)) + [B - 1],
+                   f"noalloc B={B} d={d}")
