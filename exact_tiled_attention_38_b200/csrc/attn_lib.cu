@@ -412,8 +412,17 @@ inline int decode_group_tile(int G) { return (G <= 4 || ETA_DECODE_MAX_GP == 4) 
 #ifndef ETA_DECODE_PS_HS32
 #define ETA_DECODE_PS_HS32 2
 #endif
+// The same pass for d = 64 and ETA_DECODE_PS64_MIN_G to 32 query heads per KV
+// head (0 turns it off); the CUDA-core pass reads the cache once per chunk of
+// 4 heads, so larger groups at d = 64 belong here.
+#ifndef ETA_DECODE_PS64_MIN_G
+#define ETA_DECODE_PS64_MIN_G 2
+#endif
 inline bool decode_use_ps(int G, int d) {
-  return ETA_DECODE_PS_MIN_G > 0 && d == 128 && G >= ETA_DECODE_PS_MIN_G && G <= 32;
+  if (G > 32) return false;
+  if (d == 128) return ETA_DECODE_PS_MIN_G > 0 && G >= ETA_DECODE_PS_MIN_G;
+  if (d == 64) return ETA_DECODE_PS64_MIN_G > 0 && G >= ETA_DECODE_PS64_MIN_G;
+  return false;
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -425,7 +434,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 struct PsLayout {
   size_t tok_off, tile_off, starts, part_o, part_lse, total;
 };
-inline PsLayout ps_layout(int B, int Hkv, int G, int nc, bool partials) {
+inline PsLayout ps_layout(int B, int Hkv, int G, int d, int nc, bool partials) {
   PsLayout L;
   L.tok_off = 0;
   L.tile_off = align_up(static_cast<size_t>(B) * 8, 256);
@@ -436,7 +445,7 @@ inline PsLayout ps_layout(int B, int Hkv, int G, int nc, bool partials) {
     L.starts = align_up(end, 256);
     end = L.starts + static_cast<size_t>(nc) * 16;
     L.part_o = align_up(end, 256);
-    end = L.part_o + slots * G * decode_ps::D * 4;
+    end = L.part_o + slots * G * d * 4;
     L.part_lse = align_up(end, 256);
     end = L.part_lse + slots * G * 4;
   }
@@ -486,11 +495,11 @@ int launch_decode_offsets(const int32_t* seqlens, long long* tok_off, int B, cud
 // Plan, persistent stream and gather of the d = 128 decode; `ws` holds the
 // layout `L`. seg_aligned: whole segments per CTA (L has no partials, and
 // there is nothing to gather).
-template <int NP, int GP, int HS, typename T>
+template <int NP, int GP, int HS, int D, typename T>
 int launch_decode_ps(const CUtensorMap& tq, decode_ps::PParams p, const PsLayout& L, char* ws,
                      int nc, cudaStream_t st) {
-  auto kern = decode_ps::attn_decode_persistent_kernel<NP, GP, HS, T>;
-  constexpr int smem = decode_ps::PCfg<NP>::kSmemBytes;
+  auto kern = decode_ps::attn_decode_persistent_kernel<NP, GP, HS, D, T>;
+  constexpr int smem = decode_ps::PCfg<NP, D>::kSmemBytes;
   static PerDeviceOnce attr;
   const cudaError_t attr_err = attr.run([&]() {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -501,7 +510,7 @@ int launch_decode_ps(const CUtensorMap& tq, decode_ps::PParams p, const PsLayout
   p.starts = L.starts ? reinterpret_cast<int4*>(ws + L.starts) : nullptr;
   p.part_o = L.part_o ? reinterpret_cast<float*>(ws + L.part_o) : nullptr;
   p.part_lse = L.part_lse ? reinterpret_cast<float*>(ws + L.part_lse) : nullptr;
-  decode_ps::attn_decode_plan_kernel<<<1, decode_ps::kPlanThreads, 0, st>>>(p, nc);
+  decode_ps::attn_decode_plan_kernel<D><<<1, decode_ps::kPlanThreads, 0, st>>>(p, nc);
   int rc = launch_status();
   if (rc != ATTN_OK) return rc;
   // The stream and gather kernels are launched as programmatic dependents:
@@ -524,23 +533,32 @@ int launch_decode_ps(const CUtensorMap& tq, decode_ps::PParams p, const PsLayout
   cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = 0;
-  e = cudaLaunchKernelEx(&cfg, decode_ps::attn_decode_gather_kernel<T>, p, nc);
+  e = cudaLaunchKernelEx(&cfg, decode_ps::attn_decode_gather_kernel<D, T>, p, nc);
   if (e != cudaSuccess) return cuda_fail(e);
   return launch_status();
 }
 
-// The persistent decode for d = 128: q's tensor map (rows of the G heads of
-// one KV head, box padded to NP rows), then the three kernels. `ws` must hold
-// ps_layout(B, Hkv, G, nc, !seg_aligned).
+template <int D, typename T>
+int launch_decode_ps_group(const CUtensorMap& tq, const decode_ps::PParams& p, const PsLayout& L,
+                           char* ws, int nc, cudaStream_t st) {
+  if (p.G <= 4) return launch_decode_ps<16, 4, 1, D, T>(tq, p, L, ws, nc, st);
+  if (p.G <= 8) return launch_decode_ps<16, 8, 1, D, T>(tq, p, L, ws, nc, st);
+  if (p.G <= 16) return launch_decode_ps<16, 16, 1, D, T>(tq, p, L, ws, nc, st);
+  return launch_decode_ps<32, 32, ETA_DECODE_PS_HS32, D, T>(tq, p, L, ws, nc, st);
+}
+
+// The persistent decode for d = 64 and 128: q's tensor map (rows of the G
+// heads of one KV head, box padded to NP rows), then the three kernels. `ws`
+// must hold ps_layout(B, Hkv, G, d, nc, !seg_aligned).
 template <typename T>
 int decode_ps_run(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* o,
-                  float* lse, int B, int Hq, int Hkv, float scale, int window, char* ws,
+                  float* lse, int B, int Hq, int Hkv, int d, float scale, int window, char* ws,
                   bool seg_aligned, int nc, cudaStream_t st) {
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   const int G = Hq / Hkv;
   const int NP = G <= 16 ? 16 : 32;
   CUtensorMap tq;
-  const int rc = encode_3d(&tq, q, bf16, decode_ps::D, G, static_cast<long long>(B) * Hkv,
+  const int rc = encode_3d(&tq, q, bf16, d, G, static_cast<long long>(B) * Hkv,
                            static_cast<unsigned>(NP));
   if (rc != ATTN_OK) return rc;
   decode_ps::PParams p;
@@ -558,11 +576,9 @@ int decode_ps_run(const void* q, const void* kc, const void* vc, const int32_t* 
   p.seg_aligned = seg_aligned ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
-  const PsLayout L = ps_layout(B, Hkv, G, nc, !seg_aligned);
-  if (G <= 4) return launch_decode_ps<16, 4, 1, T>(tq, p, L, ws, nc, st);
-  if (G <= 8) return launch_decode_ps<16, 8, 1, T>(tq, p, L, ws, nc, st);
-  if (G <= 16) return launch_decode_ps<16, 16, 1, T>(tq, p, L, ws, nc, st);
-  return launch_decode_ps<32, 32, ETA_DECODE_PS_HS32, T>(tq, p, L, ws, nc, st);
+  const PsLayout L = ps_layout(B, Hkv, G, d, nc, !seg_aligned);
+  return d == 128 ? launch_decode_ps_group<128, T>(tq, p, L, ws, nc, st)
+                  : launch_decode_ps_group<64, T>(tq, p, L, ws, nc, st);
 }
 
 template <int D, typename T>
@@ -656,11 +672,11 @@ int decode_run(const void* q, const void* kc, const void* vc, const int32_t* seq
   }
   if (decode_use_ps(Hq / Hkv, d)) {
     const int nc = info.sm_count;
-    const PsLayout L = ps_layout(B, Hkv, Hq / Hkv, nc, true);
+    const PsLayout L = ps_layout(B, Hkv, Hq / Hkv, d, nc, true);
     void* ws = nullptr;
     if (workspace_pool(&pool) != ATTN_OK) return ATTN_ERR_CUDA;
     if (cudaMallocFromPoolAsync(&ws, L.total, pool, st) != cudaSuccess) return ATTN_ERR_CUDA;
-    const int rc = decode_ps_run<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, scale, window,
+    const int rc = decode_ps_run<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, window,
                                     static_cast<char*>(ws), false, nc, st);
     const cudaError_t fe = cudaFreeAsync(ws, st);
     if (rc != ATTN_OK) return rc;
@@ -788,8 +804,9 @@ const char* attn_strerror(int code) {
     case ATTN_ERR_TIMEOUT:
       return "a device-side wait gave up; outputs of that launch are undefined";
     case ATTN_ERR_SCRATCH:
-      return "attn_decode_noalloc: one split-KV partial (B * Hq * (d + 1) floats) exceeds its "
-             "fixed scratch of 2,097,152 floats";
+      return "attn_decode_noalloc: one split of the CUDA-core decode pass (B * Hq * (d + 1) "
+             "floats, plus B int64 token offsets above 1024 sequences) exceeds its fixed array "
+             "of 2,097,152 floats";
     default:
       return "unknown error code";
   }
@@ -1006,11 +1023,11 @@ int decode_run_noalloc(const void* q, const void* kc, const void* vc, const int3
     // results directly.
     const int nc = info.sm_count;
     const size_t cap = kNoAllocScratchFloats * sizeof(float);
-    const bool seg_aligned = ps_layout(B, Hkv, Hq / Hkv, nc, true).total > cap;
-    if (ps_layout(B, Hkv, Hq / Hkv, nc, !seg_aligned).total > cap) return ATTN_ERR_SCRATCH;
+    const bool seg_aligned = ps_layout(B, Hkv, Hq / Hkv, d, nc, true).total > cap;
+    if (ps_layout(B, Hkv, Hq / Hkv, d, nc, !seg_aligned).total > cap) return ATTN_ERR_SCRATCH;
     float* scratch = nullptr;
     if (noalloc_scratch(&scratch) != ATTN_OK) return ATTN_ERR_CUDA;
-    return decode_ps_run<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, scale, 0,
+    return decode_ps_run<T>(q, kc, vc, seqlens, o, lse, B, Hq, Hkv, d, scale, 0,
                             reinterpret_cast<char*>(scratch), seg_aligned, nc, st);
   }
 

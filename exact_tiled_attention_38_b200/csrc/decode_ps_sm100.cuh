@@ -59,7 +59,6 @@
 namespace eta {
 namespace decode_ps {
 
-constexpr int D = 128;
 constexpr int TK = 128;  // keys per tile
 constexpr int kStages = 3;
 constexpr int kSoftWarps = 4;  // key quarters of a tile (tensor-memory lane quarters)
@@ -140,7 +139,7 @@ struct PParams {
   const int* seqlens;
   const long long* tok_off;  // [B]: token offset of sequence b in the packed cache
   const int* tile_off;       // [B + 1]: first global tile of sequence b (all its KV heads)
-  void* o;                   // [B][Hq][D], input type
+  void* o;                   // [B][Hq][D], input type (D = 64 or 128: the kernels' template)
   float* lse;                // [B][Hq] natural log, or NULL
   float* part_o;             // [slots][G][D]: normalised partial O of a cut segment
   float* part_lse;           // [slots][G]: its log-sum-exp, log2 units
@@ -173,6 +172,7 @@ __device__ __forceinline__ int first_key(int len, int window) {
 // Exclusive prefix sums over the B sequences (one CTA): token offsets of the
 // packed cache and tile offsets of the global tile order (Hkv segments of
 // ceil(keys read / 128) tiles per sequence). tile_off[B] is the total.
+template <int D>
 __global__ void __launch_bounds__(kPlanThreads) attn_decode_plan_kernel(const PParams p, int nc) {
   const int* __restrict__ seqlens = p.seqlens;
   long long* __restrict__ tok_off = const_cast<long long*>(p.tok_off);
@@ -329,14 +329,21 @@ struct Cursor {
   __device__ __forceinline__ int segment(const PParams& p) const { return b * p.Hkv + g; }
 };
 
-template <int NP>
+template <int NP, int D>
 struct PCfg {
   static_assert(NP == 16 || NP == 32, "padded group");
+  static_assert(D == 64 || D == 128, "head size");
+  static constexpr int kBoxes = D / 64;               // 128-byte-swizzled boxes per row
   static constexpr int kBoxBytes = TK * 128;          // 128 keys x 64 dims
-  static constexpr int kTileBytes = 2 * kBoxBytes;    // K or V tile (32 KB)
-  static constexpr int kStageBytes = 2 * kTileBytes;  // K tile, then V tile
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;  // K or V tile
+  // A stage holds the K tile, then the V tile. With D = 64 the product
+  // O^T += V^T P^T still runs with M = 128 (the layout of the D = 128 pass):
+  // its second 64-row half of A reads a zeroed box after the V tile, so rows
+  // 64..127 of O^T stay zero and are never stored.
+  static constexpr int kZeroBytes = D == 64 ? kBoxBytes : 0;
+  static constexpr int kStageBytes = 2 * kTileBytes + kZeroBytes;
   static constexpr int kQBox = NP * 128;              // NP rows x 64 dims (or 64 keys)
-  static constexpr int kQBuf = 2 * kQBox;             // one Q (128 dims)
+  static constexpr int kQBuf = kBoxes * kQBox;        // one Q
   static constexpr int kQOff = kStages * kStageBytes;
   static constexpr int kPBuf = 2 * kQBox;             // P^T: 2 boxes of 64 keys
   static constexpr int kPOff = kQOff + 2 * kQBuf;
@@ -347,6 +354,7 @@ struct PCfg {
   static constexpr int kCtlOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kCtlOff + 64 + 1024;  // + runtime 1024-byte alignment
   static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0 && kQBox % 1024 == 0, "swizzle atoms");
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
@@ -407,13 +415,13 @@ __device__ __forceinline__ void gather4(const float* red, float (&out)[GP], Op o
 // NP: MMA width (the group padded to 16 or 32); GP <= NP: the heads the
 // softmax processes (the group padded to 4, 8, 16 or 32); HS: softmax warps
 // per key quarter, each taking GP / HS of the heads.
-template <int NP, int GP, int HS, typename T>
+template <int NP, int GP, int HS, int D, typename T>
 __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     attn_decode_persistent_kernel(const __grid_constant__ CUtensorMap tm_q, const PParams p) {
   static_assert(GP == 4 || GP == 8 || GP == 16 || GP == 32, "softmax group");
   static_assert(GP <= NP && (GP > 16) == (NP == 32), "widths");
   static_assert(HS == 1 || (HS == 2 && GP == 32), "head split");
-  using C = PCfg<NP>;
+  using C = PCfg<NP, D>;
   using R = Roles<HS>;
   constexpr int GPT = GP / HS;  // heads per softmax thread
   const int c = blockIdx.x;
@@ -463,6 +471,15 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     tmem_relinquish();
     if (lane == 0) tma_prefetch_desc(&tm_q);
   }
+  if constexpr (C::kZeroBytes > 0) {
+    // the zeroed second half of each stage's V operand (read by the tensor core)
+    for (int i = threadIdx.x; i < kStages * C::kZeroBytes / 16; i += R::kThreads) {
+      const int st = i / (C::kZeroBytes / 16), u = i - st * (C::kZeroBytes / 16);
+      *reinterpret_cast<uint4*>(smem + st * C::kStageBytes + 2 * C::kTileBytes + u * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -496,14 +513,16 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     // no tiles for this CTA (uniform over the CTA)
   } else if (warp >= R::kProd0) {
     // ------------------------------------------------------------ producers
-    // Producer pw fills stage pw with the CTA's tiles pw, pw + 3, ... Lane l
-    // copies 16-byte unit (l % 16) of rows 2i + l / 16: each instruction reads
-    // two whole 256-byte cache rows.
+    // Producer pw fills stage pw with the CTA's tiles pw, pw + 3, ... A cache
+    // row is UPR = D / 8 units of 16 bytes; lane l copies unit l % UPR of rows
+    // RPI i + l / UPR (RPI = 32 / UPR rows per instruction): each instruction
+    // reads whole cache rows.
+    constexpr int UPR = D / 8, RPI = 32 / UPR;
     const int pw = warp - R::kProd0;
     bool ok = true;
     const uint32_t kdst = smem_u32(smem + pw * C::kStageBytes);
     const uint32_t vdst = kdst + C::kTileBytes;
-    const int u = lane & 15;
+    const int u = lane % UPR;
     for (int a = 0; a < pw && a + 1 < n; ++a) cur.next(p);  // to tile pw (if in range)
     for (int j = pw; ok && j < n; j += kStages) {
       const int use = j / kStages;
@@ -516,8 +535,8 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
       const T* vbase = reinterpret_cast<const T*>(p.vc) + head_base;
       const int t0 = cur.k0 + cur.i * TK;
 #pragma unroll 4
-      for (int i = 0; i < TK / 2; ++i) {
-        const int r = 2 * i + (lane >> 4);
+      for (int i = 0; i < TK / RPI; ++i) {
+        const int r = RPI * i + lane / UPR;
         const int key = t0 + r;
         const bool valid = key < cur.len;
         const size_t row = static_cast<size_t>(valid ? key : t0);  // t0 < len: a real row
@@ -534,7 +553,7 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     // ------------------------------------------------------------ MMA issue and Q loads
     constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
     constexpr uint32_t idesc_s = umma_idesc_f16(fmt, TK, NP, 0, 0);
-    constexpr uint32_t idesc_pv = umma_idesc_f16(fmt, D, NP, 1, 0);
+    constexpr uint32_t idesc_pv = umma_idesc_f16(fmt, 128, NP, 1, 0);  // M = 128 (zero-padded for D = 64)
     const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
     const uint32_t d_hi = static_cast<uint32_t>(dq >> 32);
     const uint32_t q_lo = static_cast<uint32_t>(dq);
@@ -544,12 +563,15 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     const uint32_t p_lo = static_cast<uint32_t>(smem_desc_sw128(smem_u32(sP), 16, 1024));
     // Q of piece k goes to buffer k % 2 (its G rows; rows G..NP-1 are zero-filled
     // by the copy as out of bounds). The first piece's Q is loaded here.
-    int nq[2] = {0, 0};  // Q loads issued per buffer
+    int nq0 = 0, nq1 = 0;  // Q loads issued per buffer (scalars: no local-memory array)
     auto load_q = [&](int buf, int seg) {
-      ++nq[buf];
+      if (buf)
+        ++nq1;
+      else
+        ++nq0;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&q_full[buf], 2 * C::kQBox);
-        for (int bx = 0; bx < 2; ++bx)
+        mbar_arrive_expect_tx(&q_full[buf], C::kQBuf);
+        for (int bx = 0; bx < C::kBoxes; ++bx)
           tma_load_3d(sQ + buf * C::kQBuf + bx * C::kQBox, &tm_q, &q_full[buf], bx * 64, 0, seg);
       }
       __syncwarp();
@@ -633,8 +655,8 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     // the abort path).
     umma_commit_w(drain);
     drain_bar(drain, 0, ctl, kSiteDrain);
-    for (int buf = 0; buf < 2; ++buf)
-      if (nq[buf] > 0) drain_bar(&q_full[buf], (nq[buf] - 1) & 1, ctl, kSiteDrain);
+    if (nq0 > 0) drain_bar(&q_full[0], (nq0 - 1) & 1, ctl, kSiteDrain);
+    if (nq1 > 0) drain_bar(&q_full[1], (nq1 - 1) & 1, ctl, kSiteDrain);
   } else {
     // ------------------------------------------------------------ softmax and epilogue
     // Warp w owns the keys of quarter q4 = w % 4 (tensor-memory lanes 32 q4 ..
@@ -705,9 +727,10 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
           rescale = true;
         }
       }
-      if (rescale && !first) {
+      if (rescale && !first && q4 * 32 < D) {
         // O^T was last written by PV(j-1) of this piece; wait for it, then
-        // scale this warp's 32 dims of its heads by their alpha.
+        // scale this warp's 32 dims of its heads by their alpha (lanes D..127
+        // of a D = 64 product hold zeros).
         if (!(ok = decode::warp_all_d(wait_bar(pv_done, (j - 1) & 1, ctl, kSitePv)))) break;
         tc_fence_after();
         uint32_t o[GPT < 16 ? 16 : GPT];
@@ -759,7 +782,7 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
 #pragma unroll
         for (int h = 0; h < GPT; ++h) {
           const int hg = h0 + h;
-          if (hg < G) {
+          if (hg < G && dim < D) {
             const float ov = tot[h] > 0.f ? __uint_as_float(o[h]) / tot[h] : 0.f;
             const float l2 = tot[h] > 0.f ? m[h] + lg2_approx(tot[h]) : -INFINITY;
             if (piece_whole) {
@@ -795,8 +818,9 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
 // equal-tile-range mode) has one partial per CTA, in slots segment + cta;
 // merge them by their log-sum-exp. Segments that lay in one CTA were written
 // by it, and empty sequences by the plan kernel; both are skipped.
-template <typename T>
+template <int D, typename T>
 __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p, int nc) {
+  constexpr int EPL = D / 32;  // output elements per lane
   griddep_wait();  // the stream kernel's partials and outputs are visible after this
   const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -820,25 +844,35 @@ __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p
   for (int cc = c0; cc <= c1; ++cc)
     if (has_tiles(cc)) mx = fmaxf(mx, p.part_lse[(seg + cc) * p.G + hh]);
   float tot = 0.f;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc[EPL] = {};
   if (mx != -INFINITY) {
     for (int cc = c0; cc <= c1; ++cc) {
       if (!has_tiles(cc)) continue;
       const long long slot = (seg + cc) * p.G + hh;
       const float wt = ex2_approx(p.part_lse[slot] - mx);
       tot += wt;
-      const float4 x = *reinterpret_cast<const float4*>(p.part_o + slot * D + lane * 4);
-      acc[0] = fmaf(wt, x.x, acc[0]);
-      acc[1] = fmaf(wt, x.y, acc[1]);
-      acc[2] = fmaf(wt, x.z, acc[2]);
-      acc[3] = fmaf(wt, x.w, acc[3]);
+      const float* x = p.part_o + slot * D + lane * EPL;
+      float xv[EPL];
+      if constexpr (EPL == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(x);
+        xv[0] = v.x, xv[1] = v.y, xv[2] = v.z, xv[3] = v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(x);
+        xv[0] = v.x, xv[1] = v.y;
+      }
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) acc[e] = fmaf(wt, xv[e], acc[e]);
     }
   }
   const float inv = tot > 0.f ? 1.f / tot : 0.f;
-  uint2 pk;
-  pk.x = decode::pack2<T>(acc[0] * inv, acc[1] * inv);
-  pk.y = decode::pack2<T>(acc[2] * inv, acc[3] * inv);
-  *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.o) + row * D + lane * 4) = pk;
+  uint32_t pk[EPL / 2];
+#pragma unroll
+  for (int e = 0; e < EPL / 2; ++e) pk[e] = decode::pack2<T>(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  T* dst = reinterpret_cast<T*>(p.o) + row * D + lane * EPL;
+  if constexpr (EPL == 4)
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+  else
+    *reinterpret_cast<uint32_t*>(dst) = pk[0];
   if (lane == 0 && p.lse != nullptr)
     p.lse[row] = tot > 0.f ? (mx + lg2_approx(tot)) * 0.69314718055994531f : -INFINITY;
 }

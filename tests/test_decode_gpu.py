@@ -173,18 +173,26 @@ def test_decode_tensor_core_single_split_writes_output(lib):
 # equal contiguous ranges, one per CTA; segments cut between CTAs are merged by
 # the gather kernel. These cases stress the cuts.
 PS_CASES = [
-    # B, Hq, Hkv, lengths, dtype
-    (1, 8, 1, [1000], BF16),                  # 8 tiles over every CTA: most CTAs own none
-    (3, 32, 2, [70000, 5, 300], BF16),        # one long segment cut over many CTAs
-    (300, 16, 2, "short", F16),               # many short sequences, empties between
-    (64, 32, 1, "ragged", BF16),              # MQA at the workload's scale
-    (64, 128, 8, "ragged", BF16),             # group 16 at the workload's scale
+    # B, Hq, Hkv, d, lengths, dtype
+    (1, 8, 1, 128, [1000], BF16),                 # 8 tiles over every CTA: most CTAs own none
+    (3, 32, 2, 128, [70000, 5, 300], BF16),       # one long segment cut over many CTAs
+    (300, 16, 2, 128, "short", F16),              # many short sequences, empties between
+    (64, 32, 1, 128, "ragged", BF16),             # MQA at the workload's scale
+    (64, 128, 8, 128, "ragged", BF16),            # group 16 at the workload's scale
+    # d = 64: the same pass with a 64-dim K tile and the P V product's upper
+    # 64 rows reading a zeroed box
+    (5, 6, 3, 64, [1, 127, 128, 129, 0], BF16),   # group 2, tile tails
+    (1, 8, 1, 64, [1000], F16),                   # group 8, most CTAs own no tile
+    (3, 32, 2, 64, [70000, 5, 300], F16),         # group 16, one segment cut over many CTAs
+    (300, 8, 2, 64, "short", BF16),               # group 4, many short sequences
+    (64, 32, 1, 64, "ragged", BF16),              # MQA at the workload's scale
+    (64, 32, 8, 64, "ragged", BF16),              # group 4 at the workload's scale
 ]
 
 
-@pytest.mark.parametrize("case", PS_CASES, ids=lambda c: f"B{c[0]}h{c[1]}kv{c[2]}")
+@pytest.mark.parametrize("case", PS_CASES, ids=lambda c: f"B{c[0]}h{c[1]}kv{c[2]}d{c[3]}")
 def test_decode_persistent_cuts(lib, case):
-    B, Hq, Hkv, lens, dt = case
+    B, Hq, Hkv, d, lens, dt = case
     if lens == "short":
         sl = workloads.decode_seqlens(B, 0, 200, 2500)
         sl[::7] = 0
@@ -192,14 +200,14 @@ def test_decode_persistent_cuts(lib, case):
         sl = workloads.decode_seqlens(B, 1024, 8192, 2501)
     else:
         sl = torch.tensor(lens, dtype=torch.int32)
-    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, 128, sl, dt,
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, d, sl, dt,
                                             seed=2600 + PS_CASES.index(case))
-    scale = 128 ** -0.5
+    scale = d ** -0.5
     o, lse = run(lib, q.to(DEV), kc.to(DEV), vc.to(DEV), sl.to(DEV), Hkv, scale)
     o2, lse2 = run(lib, q.to(DEV), kc.to(DEV), vc.to(DEV), sl.to(DEV), Hkv, scale)
     assert torch.equal(o, o2) and torch.equal(lse, lse2)  # fixed assignment: bitwise repeatable
     o_ref, lse_ref = oracle.decode_ref(q, kc, vc, sl, scale, Hkv)
-    compare(o, lse, o_ref, lse_ref, dt, f"persistent {case[:3]}")
+    compare(o, lse, o_ref, lse_ref, dt, f"persistent {case[:4]}")
 
 
 # Batches above 1024 sequences: each sequence's offset in the packed cache
@@ -208,7 +216,8 @@ def test_decode_persistent_cuts(lib, case):
 BIG_B_CASES = [
     # B, Hq, Hkv, d, dtype; lengths uniform in [0, 48], every 11th empty
     (20000, 4, 4, 128, BF16),   # MHA: CUDA-core split pass
-    (20000, 8, 2, 64, F16),     # d = 64, group 4: CUDA-core split pass
+    (20000, 4, 4, 64, F16),     # d = 64, MHA: CUDA-core split pass
+    (20000, 8, 2, 64, BF16),    # d = 64, group 4: persistent pass
     (20000, 4, 2, 96, BF16),    # d = 96: generic kernel
     (20000, 16, 2, 128, BF16),  # group 8: persistent pass
 ]

@@ -59,6 +59,7 @@ DECODE = [
     (2, 16, 2, 64, [129, 4096], 129, F16),
     (2, 8, 1, 128, [777, 20], 1, BF16),
     (5, 64, 4, 128, [9000, 0, 130, 4000, 257], 1100, BF16),  # group 16, persistent pass
+    (3, 32, 1, 64, [3000, 5, 700], 500, BF16),               # MQA, d = 64, persistent pass
 ]
 
 
