@@ -349,6 +349,38 @@ __device__ __forceinline__ float exp_tile(const float (&s)[NC], float c, float m
   return (a0 + a1) + (b0 + b1);
 }
 
+// p = 2^(s * c - m) for scores [C0, C1) of one row: P packed two per word into
+// pk (to be stored later), adding the fp32 sum of p into la / lb.
+template <typename T, int POLY8, int NC, int C0, int C1>
+__device__ __forceinline__ void exp_cols_regs(const float (&s)[NC], uint64_t c2, uint64_t nm2,
+                                              uint32_t (&pk)[(C1 - C0) / 2], uint64_t& la,
+                                              uint64_t& lb) {
+#pragma unroll
+  for (int w = 0; w < (C1 - C0) / 2; ++w) {
+    const int k = C0 + 2 * w;
+    const uint64_t x2 = f2_fma(f2_make(s[k], s[k + 1]), c2, nm2);
+    float x0, x1;
+    f2_split(x2, x0, x1);
+    const uint64_t e2 =
+        ((k & 7) < POLY8) ? ex2_poly2(x0, x1) : f2_make(ex2_approx(x0), ex2_approx(x1));
+    if (w & 1)
+      lb = f2_add(lb, e2);
+    else
+      la = f2_add(la, e2);
+    float e0, e1;
+    f2_split(e2, e0, e1);
+    pk[w] = pack2<T>(e0, e1);
+  }
+}
+
+// Own-P layout (d = 64): compute the first half of P into registers before
+// waiting for the previous P V product, which may still read P's columns,
+// then store it and compute the second half straight into tensor memory (1);
+// or wait first and write P as it is computed (0).
+#ifndef ETA_PREFILL_OWNP_LATE_WAIT
+#define ETA_PREFILL_OWNP_LATE_WAIT 1
+#endif
+
 // OUT_F32: O is written as fp32 (O / l, not rounded), for partial results
 // that are merged further (tm_o then maps an fp32 tensor with 32 x 32 boxes).
 template <int D, typename T, bool CAUSAL, bool WINDOW, int POLY8, bool PINGPONG, int SPLIT = 1,
@@ -385,7 +417,7 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
   uint64_t* s_free = x_down + 4 * NQT;  // [NQT]: the softmax has read S_t (own-P layout)
   uint64_t* pv_done = s_free + NQT;     // [NQT]: P_t V complete (own-P layout)
   constexpr bool OWNP = C::kOwnP;
-  static_assert(!OWNP || (SPLIT == 1 && !PINGPONG), "own-P layout: one thread per row");
+  static_assert(!OWNP || SPLIT == 1, "own-P layout: one thread per row");
   CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem + C::kCtlOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kCtlOff + 32);
 
@@ -793,21 +825,52 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
           l *= alpha;
         }
         const float m_use = (m == -INFINITY) ? 0.f : m;
+        if (PINGPONG && OWNP && np > 0) {
+          // Own-P with turns: wait for the previous P_t V product before
+          // taking the turn, so a turn is spent on exponentials only.
+          if (!(ok = warp_all(wait_bar(&pv_done[t], (np - 1) & 1, ctl, kSitePvDone)))) break;
+          tc_fence_after();
+        }
         if (PINGPONG) {
           if (!(ok = warp_all(wait_bar(&turn[t], tk & 1, ctl, kSiteTurn)))) break;
           ++tk;
         }
-        if (OWNP && np > 0) {
-          // P_t's columns and O_t: the previous P_t V product must be complete.
-          if (!(ok = warp_all(wait_bar(&pv_done[t], (np - 1) & 1, ctl, kSitePvDone)))) break;
-          tc_fence_after();
-        }
-        ++np;
         float lsum;
-        if (POLY8 > 0 && !edge && !wedge)
-          lsum = exp_tile<T, POLY8, NC>(s, sl2, m_use, tP);
-        else
-          lsum = exp_tile<T, 0, NC>(s, sl2, m_use, tP);
+        if constexpr (OWNP && ETA_PREFILL_OWNP_LATE_WAIT && !PINGPONG) {
+          // (the polynomial exponential option applies to the other branch only)
+          static_assert(NC == 128, "own-P rows");
+          const uint64_t c2 = f2_make(sl2, sl2);
+          const uint64_t nm2 = f2_make(-m_use, -m_use);
+          uint64_t la = f2_make(0.f, 0.f), lb = la;
+          uint32_t pa[32], pb[16];
+          exp_cols_regs<T, 0, NC, 0, 64>(s, c2, nm2, pa, la, lb);
+          if (np > 0) {
+            if (!(ok = warp_all(wait_bar(&pv_done[t], (np - 1) & 1, ctl, kSitePvDone)))) break;
+            tc_fence_after();
+          }
+          ++np;
+          tmem_st_x16(tP, *reinterpret_cast<uint32_t(*)[16]>(pa));
+          tmem_st_x16(tP + 16, *reinterpret_cast<uint32_t(*)[16]>(pa + 16));
+          exp_cols_regs<T, 0, NC, 64, 96>(s, c2, nm2, pb, la, lb);
+          tmem_st_x16(tP + 32, pb);
+          exp_cols_regs<T, 0, NC, 96, 128>(s, c2, nm2, pb, la, lb);
+          tmem_st_x16(tP + 48, pb);
+          float a0, a1, b0, b1;
+          f2_split(la, a0, a1);
+          f2_split(lb, b0, b1);
+          lsum = (a0 + a1) + (b0 + b1);
+        } else {
+          if (OWNP && !PINGPONG && np > 0) {
+            // P_t's columns and O_t: the previous P_t V product must be complete.
+            if (!(ok = warp_all(wait_bar(&pv_done[t], (np - 1) & 1, ctl, kSitePvDone)))) break;
+            tc_fence_after();
+          }
+          ++np;
+          if (POLY8 > 0 && !edge && !wedge)
+            lsum = exp_tile<T, POLY8, NC>(s, sl2, m_use, tP);
+          else
+            lsum = exp_tile<T, 0, NC>(s, sl2, m_use, tP);
+        }
         l += lsum;
         if (PINGPONG) mbar_arrive(&turn[t ^ 1]);
         if (i > s0 && __any_sync(0xffffffffu, need)) {

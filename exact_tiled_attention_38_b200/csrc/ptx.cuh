@@ -52,8 +52,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Suspend-time hint of the first poll of every bounded wait, in nanoseconds;
+// 0 selects the plain try_wait (system-dependent suspend time). Measured on
+// B200 with the plain form against a 1 ms hint: 2K causal MHA prefill 0.0819
+// against 0.0840 ms, d = 64 0.0676 against 0.0696 ms, ragged group-4 decode
+// 0.2132 against 0.2153 ms.
 #ifndef ETA_SUSPEND_HINT_NS
-#define ETA_SUSPEND_HINT_NS 1000000
+#define ETA_SUSPEND_HINT_NS 0
 #endif
 // try_wait with a suspend-time hint: the thread sleeps until the phase
 // completes (it is woken then) or the hint in nanoseconds passes. A hint of 0
