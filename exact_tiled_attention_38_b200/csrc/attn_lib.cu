@@ -225,6 +225,13 @@ int launch_fill_empty(void* o, float* lse, long long rows, int D, cudaStream_t s
 #ifndef ETA_PREFILL_POLY8
 #define ETA_PREFILL_POLY8 0
 #endif
+// The same for d = 64, whose exponential phase keeps the special-function
+// unit busy while both softmax groups of a CTA run it. Measured on B200
+// (causal 2K / non-causal 4K, d = 64): 0.0665-0.0676 / 0.373 ms without,
+// 0.0717 / 0.399 ms with 2, 0.0737 / 0.408 ms with 4, 0.0814 / 0.469 ms with 6.
+#ifndef ETA_PREFILL_POLY8_D64
+#define ETA_PREFILL_POLY8_D64 0
+#endif
 
 // Prefill kernel knob: L2 prefetch of the next item's query tiles, issued by
 // the producer right after the current item's own query loads. Measured
@@ -260,7 +267,8 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
                    const CUtensorMap& to, const prefill::Params& p, int grid, cudaStream_t st) {
   constexpr int SPLIT = D == 128 ? ETA_PREFILL_SPLIT : 1;
   constexpr bool PINGPONG = D == 64 && ETA_PREFILL_PINGPONG64;
-  auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, WINDOW, ETA_PREFILL_POLY8, PINGPONG, SPLIT,
+  constexpr int POLY8 = D == 64 ? ETA_PREFILL_POLY8_D64 : ETA_PREFILL_POLY8;
+  auto kern = prefill::attn_prefill_kernel<D, T, CAUSAL, WINDOW, POLY8, PINGPONG, SPLIT,
                                            ETA_PREFILL_PREFETCH_Q != 0, OUT_F32>;
   constexpr int smem = prefill::Cfg<D>::kSmemBytes;
   static PerDeviceOnce attr;
@@ -528,9 +536,11 @@ int launch_decode_ps(const CUtensorMap& tq, decode_ps::PParams p, const PsLayout
   p.starts = L.starts ? reinterpret_cast<int4*>(ws + L.starts) : nullptr;
   p.part_o = L.part_o ? reinterpret_cast<float*>(ws + L.part_o) : nullptr;
   p.part_lse = L.part_lse ? reinterpret_cast<float*>(ws + L.part_lse) : nullptr;
-  decode_ps::attn_decode_plan_kernel<D><<<1, decode_ps::kPlanThreads, 0, st>>>(p, nc);
-  int rc = launch_status();
-  if (rc != ATTN_OK) return rc;
+  if (!p.inline_plan) {
+    decode_ps::attn_decode_plan_kernel<D><<<1, decode_ps::kPlanThreads, 0, st>>>(p, nc);
+    const int rc = launch_status();
+    if (rc != ATTN_OK) return rc;
+  }
   // The stream and gather kernels are launched as programmatic dependents:
   // each may start before the previous kernel ends and waits on the device
   // (griddepcontrol.wait) for its results, so launch gaps overlap work.
@@ -566,6 +576,15 @@ int launch_decode_ps_group(const CUtensorMap& tq, const decode_ps::PParams& p, c
   return launch_decode_ps<32, 32, ETA_DECODE_PS_HS32, D, T>(tq, p, L, ws, nc, st);
 }
 
+// Batches of up to this many sequences skip the plan kernel: each CTA of the
+// persistent pass sums the lengths itself (one read of B lengths per CTA).
+// Measured on B200 (64 sequences of 1K-8K tokens): group 4 0.2093 against
+// 0.2112 ms with the plan kernel, group 16 0.2276 / 0.2358 ms, MQA 0.0617 /
+// 0.0638 ms; 8 sequences of 16K-32K 0.1459 / 0.1539 ms.
+#ifndef ETA_DECODE_INLINE_PLAN_MAX_B
+#define ETA_DECODE_INLINE_PLAN_MAX_B 2048
+#endif
+
 // The persistent decode for d = 64 and 128: q's tensor map (rows of the G
 // heads of one KV head, box padded to NP rows), then the three kernels. `ws`
 // must hold ps_layout(B, Hkv, G, d, nc, !seg_aligned).
@@ -593,6 +612,7 @@ int decode_ps_run(const void* q, const void* kc, const void* vc, const int32_t* 
   p.G = G;
   p.window = window;
   p.seg_aligned = seg_aligned ? 1 : 0;
+  p.inline_plan = (!seg_aligned && B <= ETA_DECODE_INLINE_PLAN_MAX_B) ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
   const PsLayout L = ps_layout(B, Hkv, G, d, nc, !seg_aligned);

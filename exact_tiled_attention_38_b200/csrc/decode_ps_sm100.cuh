@@ -186,6 +186,7 @@ struct PParams {
   int G;
   int window;       // > 0: each new token reads only the last `window` cached tokens
   int seg_aligned;  // 1: CTAs take whole segments (no partials); 0: equal tile ranges
+  int inline_plan;  // 1: no plan kernel; each CTA finds its range from seqlens (equal ranges)
   float scale_log2;
   uint64_t wait_ns;
 };
@@ -330,11 +331,11 @@ struct Cursor {
   int len, k0;        // keys read of sequence b: [k0, len)
   long long tok;      // token offset of sequence b
 
+  // Length, first key and tile count of sequence b (tok is kept by the caller).
   __device__ __forceinline__ void load_seq(const PParams& p) {
-    nt = (p.tile_off[b + 1] - p.tile_off[b]) / p.Hkv;
     len = max(p.seqlens[b], 0);
     k0 = first_key(len, p.window);
-    tok = p.tok_off[b];
+    nt = (len - k0 + TK - 1) / TK;
   }
   __device__ __forceinline__ void seek(const PParams& p, long long t) {
     int lo = 0, hi = p.B - 1;  // largest b with tile_off[b] <= t
@@ -347,6 +348,7 @@ struct Cursor {
     }
     b = lo;
     load_seq(p);
+    tok = p.tok_off[b];
     const int r = static_cast<int>(t - p.tile_off[b]);
     g = r / nt;
     i = r - g * nt;
@@ -357,10 +359,11 @@ struct Cursor {
     i = 0;
     if (++g < p.Hkv) return;
     g = 0;
-    do {
+    do {  // the next sequence with keys; token offsets move by each length
+      tok += len;
       ++b;
-    } while (b < p.B - 1 && p.tile_off[b + 1] == p.tile_off[b]);
-    load_seq(p);
+      load_seq(p);
+    } while (nt == 0 && b < p.B - 1);
   }
   __device__ __forceinline__ int segment(const PParams& p) const { return b * p.Hkv + g; }
 };
@@ -544,26 +547,118 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
   const uint32_t tO = tmem + 2 * NP;  // O^T: columns [2 NP, 3 NP)
   const int G = p.G;
 
-  // The plan is written by the kernel launched just before this one, which
-  // lets this grid start early (programmatic dependent launch): the set-up
-  // above overlaps it, and this wait returns once its writes are visible.
-  // The gather grid after this one may then start and wait in the same way.
+  // The kernel launched just before this one (the plan, or the caller's last
+  // kernel when the plan is inline) may still be running: this grid starts
+  // early (programmatic dependent launch), the set-up above overlaps it, and
+  // this wait returns once its writes are visible. The gather grid after this
+  // one may then start and wait in the same way.
   griddep_wait();
   griddep_launch_dependents();
-  const Range rg = cta_range(p, c, gridDim.x);
-  const int n = rg.hi > rg.lo ? static_cast<int>(rg.hi - rg.lo) : 0;  // tiles of this CTA
+  Range rg;
   Cursor cur;
-  if (n > 0) {
-    if (p.seg_aligned) {
-      cur.seek(p, rg.lo);
-    } else {  // the plan found this CTA's first tile
-      const int4 st = p.starts[c];
-      cur.b = st.x;
+  if (p.inline_plan) {
+    // Prefix sums over the sequences in this CTA (small batches): the total
+    // tile count, this CTA's range and its first tile, without a plan kernel.
+    // CTA 0 also writes the tile offsets the gather kernel reads, and CTA
+    // b % nc writes O = 0, LSE = -inf for an empty sequence b.
+    long long* wsum = reinterpret_cast<long long*>(red);  // [warps][2], free before the stream
+    volatile long long* start = reinterpret_cast<volatile long long*>(smem + C::kCtlOff + 40);
+    const int nthr = R::kThreads, nw = nthr / 32;
+    const int per = (p.B + nthr - 1) / nthr;
+    const int b0 = threadIdx.x * per, b1 = min(p.B, b0 + per);
+    long long til = 0, tok = 0;
+    for (int b = b0; b < b1; ++b) {
+      const int len = max(p.seqlens[b], 0);
+      tok += len;
+      til += static_cast<long long>(p.Hkv) * ((len - first_key(len, p.window) + TK - 1) / TK);
+    }
+    long long xt = til, xk = tok;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long yt = __shfl_up_sync(0xffffffffu, xt, o);
+      const long long yk = __shfl_up_sync(0xffffffffu, xk, o);
+      if (lane >= o) {
+        xt += yt;
+        xk += yk;
+      }
+    }
+    if (lane == 31) {
+      wsum[2 * warp] = xt;
+      wsum[2 * warp + 1] = xk;
+    }
+    if (threadIdx.x == 0) start[0] = -1;
+    __syncthreads();
+    if (warp == 0) {
+      long long wt = lane < nw ? wsum[2 * lane] : 0, wk = lane < nw ? wsum[2 * lane + 1] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long yt = __shfl_up_sync(0xffffffffu, wt, o);
+        const long long yk = __shfl_up_sync(0xffffffffu, wk, o);
+        if (lane >= o) {
+          wt += yt;
+          wk += yk;
+        }
+      }
+      __syncwarp();
+      if (lane < nw) {
+        wsum[2 * lane] = wt;
+        wsum[2 * lane + 1] = wk;
+      }
+    }
+    __syncthreads();
+    const long long T_all = wsum[2 * (nw - 1)];
+    long long l_run = xt - til + (warp > 0 ? wsum[2 * (warp - 1)] : 0);  // exclusive
+    long long t_run = xk - tok + (warp > 0 ? wsum[2 * (warp - 1) + 1] : 0);
+    rg.lo = c * T_all / gridDim.x;
+    rg.hi = (c + 1) * T_all / gridDim.x;
+    for (int b = b0; b < b1; ++b) {
+      const int len = max(p.seqlens[b], 0);
+      const int nt = (len - first_key(len, p.window) + TK - 1) / TK;
+      const long long span = static_cast<long long>(p.Hkv) * nt;
+      if (c == 0) const_cast<int*>(p.tile_off)[b] = static_cast<int>(l_run);
+      if (nt == 0 && b % static_cast<int>(gridDim.x) == c) {
+        for (int h = 0; h < p.Hq; ++h) {
+          const size_t row = static_cast<size_t>(b) * p.Hq + h;
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) + row * D);
+          for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (p.lse != nullptr) p.lse[row] = -INFINITY;
+        }
+      }
+      if (rg.lo < rg.hi && l_run <= rg.lo && rg.lo < l_run + span) {
+        start[0] = b;
+        start[1] = rg.lo - l_run;
+        start[2] = t_run;
+      }
+      l_run += span;
+      t_run += len;
+    }
+    if (c == 0 && threadIdx.x == 0) const_cast<int*>(p.tile_off)[p.B] = static_cast<int>(T_all);
+    __syncthreads();
+    if (start[0] < 0) rg.hi = rg.lo;  // (no tile found: cannot happen when lo < T)
+    if (rg.lo < rg.hi) {
+      cur.b = static_cast<int>(start[0]);
       cur.load_seq(p);
-      cur.g = st.y;
-      cur.i = st.z;
+      const int r = static_cast<int>(start[1]);
+      cur.g = r / cur.nt;
+      cur.i = r - cur.g * cur.nt;
+      cur.tok = start[2];
+    }
+  } else {
+    rg = cta_range(p, c, gridDim.x);
+    if (rg.hi > rg.lo) {
+      if (p.seg_aligned) {
+        cur.seek(p, rg.lo);
+      } else {  // the plan found this CTA's first tile
+        const int4 st = p.starts[c];
+        cur.b = st.x;
+        cur.load_seq(p);
+        cur.tok = p.tok_off[cur.b];
+        cur.g = st.y;
+        cur.i = st.z;
+      }
     }
   }
+  const int n = rg.hi > rg.lo ? static_cast<int>(rg.hi - rg.lo) : 0;  // tiles of this CTA
 
   if (n == 0) {
     // no tiles for this CTA (uniform over the CTA)

@@ -837,13 +837,16 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
         }
         float lsum;
         if constexpr (OWNP && ETA_PREFILL_OWNP_LATE_WAIT && !PINGPONG) {
-          // (the polynomial exponential option applies to the other branch only)
           static_assert(NC == 128, "own-P rows");
           const uint64_t c2 = f2_make(sl2, sl2);
           const uint64_t nm2 = f2_make(-m_use, -m_use);
           uint64_t la = f2_make(0.f, 0.f), lb = la;
           uint32_t pa[32], pb[16];
-          exp_cols_regs<T, 0, NC, 0, 64>(s, c2, nm2, pa, la, lb);
+          const bool poly = POLY8 > 0 && !edge && !wedge;  // unmasked tiles only
+          if (poly)
+            exp_cols_regs<T, POLY8, NC, 0, 64>(s, c2, nm2, pa, la, lb);
+          else
+            exp_cols_regs<T, 0, NC, 0, 64>(s, c2, nm2, pa, la, lb);
           if (np > 0) {
             if (!(ok = warp_all(wait_bar(&pv_done[t], (np - 1) & 1, ctl, kSitePvDone)))) break;
             tc_fence_after();
@@ -851,9 +854,15 @@ __global__ void __launch_bounds__(kernel_threads(SPLIT), 1)
           ++np;
           tmem_st_x16(tP, *reinterpret_cast<uint32_t(*)[16]>(pa));
           tmem_st_x16(tP + 16, *reinterpret_cast<uint32_t(*)[16]>(pa + 16));
-          exp_cols_regs<T, 0, NC, 64, 96>(s, c2, nm2, pb, la, lb);
+          if (poly)
+            exp_cols_regs<T, POLY8, NC, 64, 96>(s, c2, nm2, pb, la, lb);
+          else
+            exp_cols_regs<T, 0, NC, 64, 96>(s, c2, nm2, pb, la, lb);
           tmem_st_x16(tP + 32, pb);
-          exp_cols_regs<T, 0, NC, 96, 128>(s, c2, nm2, pb, la, lb);
+          if (poly)
+            exp_cols_regs<T, POLY8, NC, 96, 128>(s, c2, nm2, pb, la, lb);
+          else
+            exp_cols_regs<T, 0, NC, 96, 128>(s, c2, nm2, pb, la, lb);
           tmem_st_x16(tP + 48, pb);
           float a0, a1, b0, b1;
           f2_split(la, a0, a1);
