@@ -212,14 +212,18 @@ def test_decode_persistent_cuts(lib, case):
 
 # Batches above 1024 sequences: each sequence's offset in the packed cache
 # comes from one prefix-sum kernel per call (the plan kernel on the persistent
-# pass) instead of each CTA summing the lengths before its own.
+# pass above 2048 sequences) instead of each CTA summing the lengths before its
+# own; up to 2048 sequences the persistent pass's CTAs scan the lengths
+# themselves (several per thread at 2048).
 BIG_B_CASES = [
     # B, Hq, Hkv, d, dtype; lengths uniform in [0, 48], every 11th empty
     (20000, 4, 4, 128, BF16),   # MHA: CUDA-core split pass
     (20000, 4, 4, 64, F16),     # d = 64, MHA: CUDA-core split pass
     (20000, 8, 2, 64, BF16),    # d = 64, group 4: persistent pass
     (20000, 4, 2, 96, BF16),    # d = 96: generic kernel
-    (20000, 16, 2, 128, BF16),  # group 8: persistent pass
+    (20000, 16, 2, 128, BF16),  # group 8: persistent pass (plan kernel)
+    (2048, 16, 2, 128, BF16),   # group 8: the largest batch whose CTAs find their ranges themselves
+    (2048, 32, 1, 64, F16),     # MQA, d = 64, the same
 ]
 
 
