@@ -1,5 +1,5 @@
 // Exact attention, decode, as one persistent streaming pass on the tensor
-// cores (sm_100a), head size 128, up to 32 query heads per KV head.
+// cores (sm_100a), head size 64 or 128, 2 to 32 query heads per KV head.
 //
 // Generating a token re-reads the whole KV cache of its sequence (first page,
 // the token-generation case; zimaspace page, "Reduced IO Is Not the Same as
@@ -14,20 +14,22 @@
 // writes either the result itself (the whole segment lay in its range) or a
 // normalised partial with its log-sum-exp, which the gather kernel merges.
 //
-// Three kernels per call:
-//   attn_decode_plan_kernel        one CTA: per sequence, token offset in the
-//                                  packed cache (int64) and tile offset in the
-//                                  global tile order (int32 prefix over
-//                                  sequences, KV heads included); each CTA's
-//                                  first tile position; O = 0, LSE = -inf for
-//                                  empty sequences
-//   attn_decode_persistent_kernel  the stream (below)
+// Two or three kernels per call:
+//   attn_decode_plan_kernel        (batches above 2048 sequences, and the
+//                                  whole-segment mode) one CTA: per sequence,
+//                                  token offset in the packed cache (int64)
+//                                  and tile offset in the global tile order
+//                                  (int32 prefix over sequences, KV heads
+//                                  included); each CTA's first tile position;
+//                                  O = 0, LSE = -inf for empty sequences
+//   attn_decode_persistent_kernel  the stream (below); for smaller batches
+//                                  each CTA forms the same prefix sums itself
 //   attn_decode_gather_kernel      one warp per (sequence, query head) of a
 //                                  segment cut between CTAs: merges its
 //                                  partials by their log-sum-exp
 //
 // Per tile (G query heads of KV head g, padded to NP = 16 or 32):
-//   S^T = K_j Q^T      M = 128 keys, N = NP, K = 128 dims; A = K tile
+//   S^T = K_j Q^T      M = 128 keys, N = NP, K = D dims; A = K tile
 //                      (K-major), B = Q (K-major); fp32 in tensor memory,
 //                      lane = key, column = head (two buffers)
 //   softmax            warp w owns keys 32w..32w+31; per head the tile max by
@@ -36,15 +38,17 @@
 //                      per head; P^T [head][key] rounded to the input type in
 //                      shared memory (two buffers); l kept per key slot
 //   O^T += V_j^T P^T   M = 128 dims, N = NP, K = 128 keys; A = the V tile read
-//                      MN-major, B = P^T (K-major); fp32 in tensor memory
+//                      MN-major (for D = 64 its upper 64 rows read a zeroed
+//                      box), B = P^T (K-major); fp32 in tensor memory
 // Q of each segment comes in by TMA (two buffers, the next segment's Q loaded
 // while the current one runs); K and V by 16-byte cp.async straight into the
 // 128-byte-swizzled layout, zero-filled past the segment's last key (the
 // packed cache's extent is only known on the device).
 //
-// Warp roles (256 threads): warps 0-3 softmax and epilogue, warp 4 tensor
-// memory owner, MMA issue and Q loads (whole warp, one elected lane), warps
-// 5-7 producers, each owning one 64 KB ring stage. Every wait is bounded.
+// Warp roles (HS softmax warps per key quarter): warps 0 .. 4 HS - 1 softmax
+// and epilogue, then the tensor memory owner (MMA issue and Q loads, whole
+// warp, one elected lane), then three producers, each owning one ring stage.
+// Every wait is bounded.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -1019,31 +1023,54 @@ __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p
   if (c0 == c1) return;
   const long long seg = static_cast<long long>(b) * p.Hkv + g;
   // CTAs between c0 and c1 with an empty tile range (fewer tiles than CTAs)
-  // wrote nothing: their slots are skipped.
+  // wrote nothing: their slots are skipped. The partials of the first kMaxP
+  // CTAs are all loaded before any is used, so their loads overlap; a
+  // running maximum then folds them (and, for longer cuts, the rest) in.
   auto has_tiles = [&](int cc) { return cc * T_all / nc < (cc + 1) * T_all / nc; };
-  float mx = -INFINITY;
-  for (int cc = c0; cc <= c1; ++cc)
-    if (has_tiles(cc)) mx = fmaxf(mx, p.part_lse[(seg + cc) * p.G + hh]);
-  float tot = 0.f;
-  float acc[EPL] = {};
-  if (mx != -INFINITY) {
-    for (int cc = c0; cc <= c1; ++cc) {
-      if (!has_tiles(cc)) continue;
+  constexpr int kMaxP = 6;
+  float lse_r[kMaxP], xv[kMaxP][EPL];
+#pragma unroll
+  for (int k = 0; k < kMaxP; ++k) {
+    const int cc = c0 + k;
+    lse_r[k] = -INFINITY;
+    if (cc <= c1 && has_tiles(cc)) {
       const long long slot = (seg + cc) * p.G + hh;
-      const float wt = ex2_approx(p.part_lse[slot] - mx);
-      tot += wt;
+      lse_r[k] = p.part_lse[slot];
       const float* x = p.part_o + slot * D + lane * EPL;
-      float xv[EPL];
       if constexpr (EPL == 4) {
         const float4 v = *reinterpret_cast<const float4*>(x);
-        xv[0] = v.x, xv[1] = v.y, xv[2] = v.z, xv[3] = v.w;
+        xv[k][0] = v.x, xv[k][1] = v.y, xv[k][2] = v.z, xv[k][3] = v.w;
       } else {
         const float2 v = *reinterpret_cast<const float2*>(x);
-        xv[0] = v.x, xv[1] = v.y;
+        xv[k][0] = v.x, xv[k][1] = v.y;
       }
+    } else {
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) acc[e] = fmaf(wt, xv[e], acc[e]);
+      for (int e = 0; e < EPL; ++e) xv[k][e] = 0.f;
     }
+  }
+  float mx = -INFINITY, tot = 0.f;
+  float acc[EPL] = {};
+  auto fold = [&](float lse, const float (&x)[EPL]) {
+    if (lse == -INFINITY) return;
+    const float nm = fmaxf(mx, lse);
+    const float sc = ex2_approx(mx - nm);  // mx = -inf gives 0
+    const float wt = ex2_approx(lse - nm);
+    tot = tot * sc + wt;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(wt, x[e], acc[e] * sc);
+    mx = nm;
+  };
+#pragma unroll
+  for (int k = 0; k < kMaxP; ++k) fold(lse_r[k], xv[k]);
+  for (int cc = c0 + kMaxP; cc <= c1; ++cc) {
+    if (!has_tiles(cc)) continue;
+    const long long slot = (seg + cc) * p.G + hh;
+    const float* x = p.part_o + slot * D + lane * EPL;
+    float xr[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) xr[e] = x[e];
+    fold(p.part_lse[slot], xr);
   }
   const float inv = tot > 0.f ? 1.f / tot : 0.f;
   uint32_t pk[EPL / 2];
