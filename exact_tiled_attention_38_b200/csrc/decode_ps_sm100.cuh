@@ -324,9 +324,17 @@ __device__ __forceinline__ Range cta_range(const PParams& p, int c, int nc) {
   return r;
 }
 
+// n / d for 0 <= n, 0 < d: a 32-bit division when both fit (the usual case;
+// a 64-bit division is a long instruction sequence on the GPU).
+__host__ __device__ __forceinline__ long long div_nonneg(long long n, long long d) {
+  if (((n | d) >> 31) == 0)
+    return static_cast<long long>(static_cast<unsigned>(n) / static_cast<unsigned>(d));
+  return n / d;
+}
+
 // The CTA whose equal tile range holds global tile t (tile-balanced mode).
 __host__ __device__ __forceinline__ int cta_of(long long t, long long T, int nc) {
-  return static_cast<int>(((t + 1) * nc - 1) / T);
+  return static_cast<int>(div_nonneg((t + 1) * nc - 1, T));
 }
 
 // Position of a global tile: sequence b, KV head g, tile i of nt in the segment.
@@ -391,9 +399,10 @@ struct PCfg {
   static constexpr int kPBuf = 2 * kQBox;             // P^T: 2 boxes of 64 keys
   static constexpr int kPOff = kQOff + 2 * kQBuf;
   static constexpr int kRedOff = kPOff + 2 * kPBuf;   // [2][warps][NP] floats
-  // full[S], empty[S], s_ready[2], p_ready[2], x_bar[2], q_full[2], q_free[2], pv_done, drain
+  // full[S], empty[S], s_ready[2], p_ready[2], x_bar[2], q_full[2], q_free[2], pv_done[2],
+  // drain, first_issued[2], full_v[S], empty_v[S]
   static constexpr int kBarOff = kRedOff + 2 * kSoftWarps * NP * 4;
-  static constexpr int kNumBars = 2 * kStages + 10 + 2 + 2;  // + first_issued[2]
+  static constexpr int kNumBars = 4 * kStages + 10 + 3 + 2;
   static constexpr int kCtlOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kCtlOff + 64 + 1024;  // + runtime 1024-byte alignment
   static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0 && kQBox % 1024 == 0, "swizzle atoms");
@@ -420,9 +429,26 @@ __device__ __forceinline__ float warp_max_redux(float x) {
 #define ETA_DECODE_PS_STAGGER 1
 #endif
 
+// A stage's K tile is released when the score product has read it and its V
+// tile when the P V product has, each loaded on its own barrier, so the next
+// K copies start while this tile's softmax runs (1); or the stage is released
+// and loaded as a whole (0).
+#ifndef ETA_DECODE_PS_KV_SPLIT
+#define ETA_DECODE_PS_KV_SPLIT 1
+#endif
+
 // Per-tile head maxima by redux.sync (1) or by the shuffle reduce-scatter (0).
 #ifndef ETA_DECODE_PS_REDUX
 #define ETA_DECODE_PS_REDUX 0
+#endif
+
+// After a piece's first tile, the softmax warps first vote (one flag per
+// warp through the exchange) on whether any score of the tile lies more than
+// the rescale threshold above its head's running maximum; only then are the
+// tile maxima reduced and exchanged (1). Or always exchange the maxima (0).
+// Both keep the same running maxima, so the results are identical.
+#ifndef ETA_DECODE_PS_VOTE
+#define ETA_DECODE_PS_VOTE 1
 #endif
 
 struct MaxOp {
@@ -512,9 +538,16 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
   uint64_t* x_bar = p_ready + 2;
   uint64_t* q_full = x_bar + 2;
   uint64_t* q_free = q_full + 2;
+  // pv_done[j % 2] completes once per product PV(j) of the tiles j of that
+  // parity: a softmax thread that waits for PV(j) knows PV(j - 2) is done (its
+  // S(j) followed it), so the phase it waits for is never ambiguous, whether
+  // or not PV(j - 1) has run yet.
   uint64_t* pv_done = q_free + 2;
-  uint64_t* drain = pv_done + 1;
+  uint64_t* drain = pv_done + 2;
   uint64_t* first_issued = drain + 1;  // producer p -> p + 1: its first stage's copies are issued
+  // With the K/V split, full / empty track a stage's K tile and these its V tile.
+  uint64_t* full_v = first_issued + 2;
+  uint64_t* empty_v = full_v + kStages;
   CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem + C::kCtlOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kCtlOff + 32);
 
@@ -525,6 +558,8 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 32);  // one cp.async arrival per producer lane
       mbar_init(&empty[s], 1);
+      mbar_init(&full_v[s], 32);
+      mbar_init(&empty_v[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_ready[i], 1);
@@ -533,7 +568,8 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_free[i], 1);
     }
-    mbar_init(pv_done, 1);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     mbar_init(drain, 1);
     mbar_init(&first_issued[0], 1);
     mbar_init(&first_issued[1], 1);
@@ -625,8 +661,8 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     const long long T_all = wsum[2 * (nw - 1)];
     long long l_run = xt - til + (warp > 0 ? wsum[2 * (warp - 1)] : 0);  // exclusive
     long long t_run = xk - tok + (warp > 0 ? wsum[2 * (warp - 1) + 1] : 0);
-    rg.lo = c * T_all / gridDim.x;
-    rg.hi = (c + 1) * T_all / gridDim.x;
+    rg.lo = div_nonneg(c * T_all, gridDim.x);
+    rg.hi = div_nonneg((c + 1) * T_all, gridDim.x);
     for (int b = b0; b < b1; ++b) {
       const int len = max(p.seqlens[b], 0);
       const int nt = (len - first_key(len, p.window) + TK - 1) / TK;
@@ -704,18 +740,44 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
       const T* kbase = reinterpret_cast<const T*>(p.kc) + head_base;
       const T* vbase = reinterpret_cast<const T*>(p.vc) + head_base;
       const int t0 = cur.k0 + cur.i * TK;
+      if constexpr (ETA_DECODE_PS_KV_SPLIT) {
+        // K, then (once PV(j - 3) has read the stage's V tile) V; each
+        // arrival fires when all this lane's earlier copies have landed.
 #pragma unroll 4
-      for (int i = 0; i < TK / RPI; ++i) {
-        const int r = RPI * i + lane / UPR;
-        const int key = t0 + r;
-        const bool valid = key < cur.len;
-        const size_t row = static_cast<size_t>(valid ? key : t0);  // t0 < len: a real row
-        const uint32_t nb = valid ? 16u : 0u;                     // 0: zero-fill, no read
-        const uint32_t off = sw128_off(r, u, C::kBoxBytes);
-        cp_async16(kdst + off, kbase + row * D + u * 8, nb);
-        cp_async16(vdst + off, vbase + row * D + u * 8, nb);
+        for (int i = 0; i < TK / RPI; ++i) {
+          const int r = RPI * i + lane / UPR;
+          const int key = t0 + r;
+          const bool valid = key < cur.len;
+          const size_t row = static_cast<size_t>(valid ? key : t0);  // t0 < len: a real row
+          cp_async16(kdst + sw128_off(r, u, C::kBoxBytes), kbase + row * D + u * 8, valid ? 16u : 0u);
+        }
+        cp_async_mbar_arrive_noinc(&full[pw]);
+        if (use > 0 &&
+            !(ok = decode::warp_all_d(wait_bar_spin(&empty_v[pw], (use - 1) & 1, ctl, kSiteEmpty))))
+          break;
+#pragma unroll 4
+        for (int i = 0; i < TK / RPI; ++i) {
+          const int r = RPI * i + lane / UPR;
+          const int key = t0 + r;
+          const bool valid = key < cur.len;
+          const size_t row = static_cast<size_t>(valid ? key : t0);
+          cp_async16(vdst + sw128_off(r, u, C::kBoxBytes), vbase + row * D + u * 8, valid ? 16u : 0u);
+        }
+        cp_async_mbar_arrive_noinc(&full_v[pw]);
+      } else {
+#pragma unroll 4
+        for (int i = 0; i < TK / RPI; ++i) {
+          const int r = RPI * i + lane / UPR;
+          const int key = t0 + r;
+          const bool valid = key < cur.len;
+          const size_t row = static_cast<size_t>(valid ? key : t0);  // t0 < len: a real row
+          const uint32_t nb = valid ? 16u : 0u;                     // 0: zero-fill, no read
+          const uint32_t off = sw128_off(r, u, C::kBoxBytes);
+          cp_async16(kdst + off, kbase + row * D + u * 8, nb);
+          cp_async16(vdst + off, vbase + row * D + u * 8, nb);
+        }
+        cp_async_mbar_arrive_noinc(&full[pw]);
       }
-      cp_async_mbar_arrive_noinc(&full[pw]);
       if (ETA_DECODE_PS_STAGGER && use == 0 && pw + 1 < kStages) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&first_issued[pw]);
@@ -785,6 +847,7 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
             umma_ss_w<1>(tS, desc_words(kd + ko, d_hi), desc_words(qd + qo, d_hi), idesc_s);
         }
         umma_commit_w(&s_ready[j & 1]);
+        if (ETA_DECODE_PS_KV_SPLIT) umma_commit_w(&empty[st]);  // K tile read
         if (last) umma_commit_w(&q_free[qb]);  // Q buffer free once this product is done
         if (first && j + (cur.nt - cur.i) < n) {
           // Load the next piece's Q into the other buffer, which piece k - 1
@@ -803,6 +866,10 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
         const int st = jp % kStages;
         if (!(ok = decode::warp_all_d(wait_bar_spin(&p_ready[jp & 1], (jp >> 1) & 1, ctl, kSiteP))))
           break;
+        if (ETA_DECODE_PS_KV_SPLIT &&
+            !(ok = decode::warp_all_d(
+                  wait_bar_spin(&full_v[st], (jp / kStages) & 1, ctl, kSiteFull))))
+          break;
         fence_proxy_async_smem();
         tc_fence_after();
         const uint32_t vd = v_lo + ((st * C::kStageBytes) >> 4);
@@ -816,8 +883,8 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
           else
             umma_ss_w<1>(tO, desc_words(vd + vo, d_hi), desc_words(pd + po, d_hi), idesc_pv);
         }
-        umma_commit_w(&empty[st]);
-        umma_commit_w(pv_done);
+        umma_commit_w(ETA_DECODE_PS_KV_SPLIT ? &empty_v[st] : &empty[st]);
+        umma_commit_w(&pv_done[jp & 1]);
       }
       if (j < n) {
         prev_first = (j == 0) || (cur.i == 0);
@@ -879,27 +946,57 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
         s[h] = (valid && h0 + h < G) ? __uint_as_float(r[h]) * sl2 : -INFINITY;
         wm[h] = s[h];
       }
-      // tile max per head: this warp's 32 keys by a reduce-scatter (lane l ends
-      // with head h0 + l % GPT), then the four key quarters through shared memory
       float* rb = red + (xc & 1) * (kSoftWarps * NP);
-      if constexpr (ETA_DECODE_PS_REDUX != 0) {
+      bool exch = true;  // exchange the tile maxima
+      if (ETA_DECODE_PS_VOTE && !first) {
+        // Vote: does any score of the tile lie more than the threshold above
+        // its head's running maximum? If not, no maximum moves (alpha = 1).
+        bool up = false;
 #pragma unroll
-        for (int h = 0; h < GPT; ++h) wm[h] = warp_max_redux(wm[h]);
-        if (lane == 0) {
-          float4* dst = reinterpret_cast<float4*>(rb + q4 * NP + h0);
+        for (int h = 0; h < GPT; ++h) up = up || (s[h] > m[h] + kRescaleThreshold);
+        up = __any_sync(0xffffffffu, up);
+        if (lane == 0) reinterpret_cast<uint32_t*>(rb)[warp] = up ? 1u : 0u;
+        mbar_arrive(&x_bar[xc & 1]);
+        if (!(ok = decode::warp_all_d(wait_bar_spin(&x_bar[xc & 1], (xc >> 1) & 1, ctl, kSiteX))))
+          break;
+        ++xc;
+        const uint4* f4 = reinterpret_cast<const uint4*>(rb);
+        uint32_t any = 0;
 #pragma unroll
-          for (int v4 = 0; v4 < GPT / 4; ++v4)
-            dst[v4] = make_float4(wm[4 * v4], wm[4 * v4 + 1], wm[4 * v4 + 2], wm[4 * v4 + 3]);
+        for (int v4 = 0; v4 < R::kSoft / 4; ++v4) {
+          const uint4 f = f4[v4];
+          any |= f.x | f.y | f.z | f.w;
         }
-      } else {
-        const float wmax = reduce_scatter<GPT>(wm, lane, MaxOp());
-        if (lane < GPT) rb[q4 * NP + h0 + lane] = wmax;
+        exch = any != 0;
+        rb = red + (xc & 1) * (kSoftWarps * NP);
       }
-      mbar_arrive(&x_bar[xc & 1]);
-      if (!(ok = decode::warp_all_d(wait_bar_spin(&x_bar[xc & 1], (xc >> 1) & 1, ctl, kSiteX)))) break;
-      ++xc;
       float tm[GPT];
-      gather4<GPT, NP>(rb + h0, tm, MaxOp());
+      if (exch) {
+        // tile max per head: this warp's 32 keys by a reduce-scatter (lane l
+        // ends with head h0 + l % GPT), then the four key quarters through
+        // shared memory
+        if constexpr (ETA_DECODE_PS_REDUX != 0) {
+#pragma unroll
+          for (int h = 0; h < GPT; ++h) wm[h] = warp_max_redux(wm[h]);
+          if (lane == 0) {
+            float4* dst = reinterpret_cast<float4*>(rb + q4 * NP + h0);
+#pragma unroll
+            for (int v4 = 0; v4 < GPT / 4; ++v4)
+              dst[v4] = make_float4(wm[4 * v4], wm[4 * v4 + 1], wm[4 * v4 + 2], wm[4 * v4 + 3]);
+          }
+        } else {
+          const float wmax = reduce_scatter<GPT>(wm, lane, MaxOp());
+          if (lane < GPT) rb[q4 * NP + h0 + lane] = wmax;
+        }
+        mbar_arrive(&x_bar[xc & 1]);
+        if (!(ok = decode::warp_all_d(wait_bar_spin(&x_bar[xc & 1], (xc >> 1) & 1, ctl, kSiteX))))
+          break;
+        ++xc;
+        gather4<GPT, NP>(rb + h0, tm, MaxOp());
+      } else {
+#pragma unroll
+        for (int h = 0; h < GPT; ++h) tm[h] = -INFINITY;
+      }
       float alpha[GPT];
       bool rescale = false;
 #pragma unroll
@@ -916,7 +1013,9 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
         // O^T was last written by PV(j-1) of this piece; wait for it, then
         // scale this warp's 32 dims of its heads by their alpha (lanes D..127
         // of a D = 64 product hold zeros).
-        if (!(ok = decode::warp_all_d(wait_bar_spin(pv_done, (j - 1) & 1, ctl, kSitePv)))) break;
+        if (!(ok = decode::warp_all_d(
+                  wait_bar_spin(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ctl, kSitePv))))
+          break;
         tc_fence_after();
         uint32_t o[TW];
         tmem_ld_np<(TW)>(tO + lane_off + h0, o);
@@ -957,7 +1056,8 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
         ++xc;
         float tot[GPT];
         gather4<GPT, NP>(rl + h0, tot, AddOp());
-        if (!(ok = decode::warp_all_d(wait_bar_spin(pv_done, j & 1, ctl, kSitePv)))) break;
+        if (!(ok = decode::warp_all_d(wait_bar_spin(&pv_done[j & 1], (j >> 1) & 1, ctl, kSitePv))))
+          break;
         tc_fence_after();
         uint32_t o[TW];
         tmem_ld_np<(TW)>(tO + lane_off + h0, o);
@@ -1010,7 +1110,7 @@ __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p
   const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= static_cast<long long>(p.B) * p.Hq) return;
-  const int b = static_cast<int>(row / p.Hq);
+  const int b = static_cast<int>(div_nonneg(row, p.Hq));
   const int h = static_cast<int>(row - static_cast<long long>(b) * p.Hq);
   const int g = h / p.G;
   const int hh = h - g * p.G;
@@ -1022,11 +1122,15 @@ __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p
   const int c1 = cta_of(a + nt - 1, T_all, nc);
   if (c0 == c1) return;
   const long long seg = static_cast<long long>(b) * p.Hkv + g;
-  // CTAs between c0 and c1 with an empty tile range (fewer tiles than CTAs)
-  // wrote nothing: their slots are skipped. The partials of the first kMaxP
-  // CTAs are all loaded before any is used, so their loads overlap; a
-  // running maximum then folds them (and, for longer cuts, the rest) in.
-  auto has_tiles = [&](int cc) { return cc * T_all / nc < (cc + 1) * T_all / nc; };
+  // CTAs between c0 and c1 with an empty tile range (possible only with
+  // fewer tiles than CTAs) wrote nothing: their slots are skipped. The
+  // partials of the first kMaxP CTAs are all loaded before any is used, so
+  // their loads overlap; a running maximum then folds them (and, for longer
+  // cuts, the rest) in.
+  const bool all_have = T_all >= nc;
+  auto has_tiles = [&](int cc) {
+    return all_have || div_nonneg(cc * T_all, nc) < div_nonneg((cc + 1) * T_all, nc);
+  };
   constexpr int kMaxP = 6;
   float lse_r[kMaxP], xv[kMaxP][EPL];
 #pragma unroll
