@@ -7,8 +7,9 @@ group of 3 (padded to 4), group 8, d = 64 and fp16, a single long sequence
 spread over many splits; for the persistent tensor-core pass (groups of 2 to
 32 with d = 128), tile tails, padded groups, MQA, the workload's scale with
 groups of 8, keys that move the running maximum at every tile, and segments
-cut between CTAs; and batches of twenty thousand short sequences, whose token
-offsets come from one prefix sum per call, on every decode path.
+cut between CTAs; bitwise repeatability of the persistent pass over many calls
+on ragged workloads; and batches of twenty thousand short sequences, whose
+token offsets come from one prefix sum per call, on every decode path.
 """
 import numpy as np
 import pytest
@@ -208,6 +209,33 @@ def test_decode_persistent_cuts(lib, case):
     assert torch.equal(o, o2) and torch.equal(lse, lse2)  # fixed assignment: bitwise repeatable
     o_ref, lse_ref = oracle.decode_ref(q, kc, vc, sl, scale, Hkv)
     compare(o, lse, o_ref, lse_ref, dt, f"persistent {case[:4]}")
+
+
+# Repeated calls on the same inputs must give bitwise-identical outputs: the
+# persistent pass's tile assignment is fixed, so any difference is a race
+# (for instance an end-of-piece wait that passes before the last P V product
+# has run). Ragged workloads at full scale, where the K/V copies, the softmax
+# and the products overlap the most.
+REPEAT_CASES = [
+    # B, Hq, Hkv, d, dtype
+    (64, 32, 8, 128, BF16),   # group 4 (the bench's decode workload shape)
+    (64, 64, 8, 128, BF16),   # group 8
+    (64, 32, 8, 64, BF16),    # group 4, d = 64
+    (64, 32, 1, 128, F16),    # MQA
+]
+
+
+@pytest.mark.parametrize("case", REPEAT_CASES, ids=lambda c: f"B{c[0]}h{c[1]}kv{c[2]}d{c[3]}")
+def test_decode_persistent_repeatable(lib, case):
+    B, Hq, Hkv, d, dt = case
+    sl = workloads.decode_seqlens(B, 1024, 8192, 2800 + REPEAT_CASES.index(case))
+    q, kc, vc, sl = workloads.random_decode(B, Hq, Hkv, d, sl, dt,
+                                            seed=2810 + REPEAT_CASES.index(case), device=DEV)
+    scale = d ** -0.5
+    o1, l1 = run(lib, q, kc, vc, sl, Hkv, scale)
+    for _ in range(12):
+        o, l = run(lib, q, kc, vc, sl, Hkv, scale)
+        assert torch.equal(o, o1) and torch.equal(l, l1), f"decode {case[:4]}: outputs differ"
 
 
 # Batches above 1024 sequences: each sequence's offset in the packed cache
