@@ -429,11 +429,15 @@ inline int decode_group_tile(int G) { return (G <= 4 || ETA_DECODE_MAX_GP == 4) 
 // thread takes GP / HS of the heads of its key, at least 8 when HS > 1).
 // Measured on B200 (64 sequences of 1K-8K tokens, median of 30 launches):
 // groups of 16 at d = 64 0.1846 ms with 2 warps per quarter against 0.2174 ms
-// with 1, at d = 128 0.2379 against 0.2358 ms (so 2 only for d = 64); groups
-// of 32 (MQA) 0.0658 / 0.0515 ms with 4 against 0.0679 / 0.0556 ms with 2 at
+// with 1; at d = 128 0.2379 against 0.2358 ms before the K/V split and the
+// tile-max vote, 0.1948-0.1969 against 0.2051 ms after them; groups of 32
+// (MQA) 0.0658 / 0.0515 ms with 4 against 0.0679 / 0.0556 ms with 2 at
 // d = 128 / 64.
 #ifndef ETA_DECODE_PS_HS16_D64
 #define ETA_DECODE_PS_HS16_D64 2
+#endif
+#ifndef ETA_DECODE_PS_HS16_D128
+#define ETA_DECODE_PS_HS16_D128 2
 #endif
 #ifndef ETA_DECODE_PS_HS32
 #define ETA_DECODE_PS_HS32 4
@@ -572,7 +576,8 @@ int launch_decode_ps_group(const CUtensorMap& tq, const decode_ps::PParams& p, c
   if (p.G <= 4) return launch_decode_ps<16, 4, 1, D, T>(tq, p, L, ws, nc, st);
   if (p.G <= 8) return launch_decode_ps<16, 8, 1, D, T>(tq, p, L, ws, nc, st);
   if (p.G <= 16)
-    return launch_decode_ps<16, 16, D == 64 ? ETA_DECODE_PS_HS16_D64 : 1, D, T>(tq, p, L, ws, nc, st);
+    return launch_decode_ps<16, 16, D == 64 ? ETA_DECODE_PS_HS16_D64 : ETA_DECODE_PS_HS16_D128, D, T>(
+        tq, p, L, ws, nc, st);
   return launch_decode_ps<32, 32, ETA_DECODE_PS_HS32, D, T>(tq, p, L, ws, nc, st);
 }
 

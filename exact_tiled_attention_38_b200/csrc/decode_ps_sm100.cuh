@@ -423,10 +423,13 @@ __device__ __forceinline__ float warp_max_redux(float x) {
 // Producers issue their first stages one after another (1), so that the
 // first tile's bytes are not interleaved with the second and third stages'
 // in the memory system, or all at once (0). Measured on B200 (64 sequences of
-// 1K-8K tokens): group 4 0.2072 against 0.2092 ms, MQA 0.0597 / 0.0618 ms,
-// group 4 at d = 64 0.1437 / 0.1478 ms.
+// 1K-8K tokens): with whole stages released at once, 1 was faster (group 4
+// 0.2072 against 0.2092 ms, MQA 0.0597 / 0.0618 ms); with K and V released
+// separately, 0 is (group 4 0.1989-0.2009 against 0.2030 ms, group 8 0.2010
+// / 0.2046 ms, 512-sequence MQA 0.2194 / 0.2235 ms, group 16 at d = 64
+// 0.1580 / 0.1600 ms; MQA equal; 256 short sequences 0.1170 / 0.1150 ms).
 #ifndef ETA_DECODE_PS_STAGGER
-#define ETA_DECODE_PS_STAGGER 1
+#define ETA_DECODE_PS_STAGGER 0
 #endif
 
 // A stage's K tile is released when the score product has read it and its V
