@@ -590,6 +590,22 @@ int launch_decode_ps_group(const CUtensorMap& tq, const decode_ps::PParams& p, c
 #define ETA_DECODE_INLINE_PLAN_MAX_B 2048
 #endif
 
+// Cost of a segment start, in tiles, when the persistent pass's CTAs split
+// the work among themselves (batches of up to ETA_DECODE_INLINE_PLAN_MAX_B
+// sequences): a CTA that starts more pieces then takes fewer tiles. Groups of
+// 9 to 16 and of 17 to 32 query heads; smaller groups split by tiles alone
+// (their softmax step is short, so a piece costs little more than its tiles).
+// Measured on B200 (64 sequences of 1K-8K tokens) against equal tile shares:
+// group 16 at d = 64 0.1477-0.1497 against 0.1581-0.1600 ms, MQA at d = 64
+// 0.0412-0.0418 / 0.0433 ms with 3 (0.0433 with 2); group 16 and MQA at
+// d = 128 and 512-sequence MQA equal.
+#ifndef ETA_DECODE_PS_SEG_COST16
+#define ETA_DECODE_PS_SEG_COST16 2
+#endif
+#ifndef ETA_DECODE_PS_SEG_COST32
+#define ETA_DECODE_PS_SEG_COST32 3
+#endif
+
 // The persistent decode for d = 64 and 128: q's tensor map (rows of the G
 // heads of one KV head, box padded to NP rows), then the three kernels. `ws`
 // must hold ps_layout(B, Hkv, G, d, nc, !seg_aligned).
@@ -618,6 +634,10 @@ int decode_ps_run(const void* q, const void* kc, const void* vc, const int32_t* 
   p.window = window;
   p.seg_aligned = seg_aligned ? 1 : 0;
   p.inline_plan = (!seg_aligned && B <= ETA_DECODE_INLINE_PLAN_MAX_B) ? 1 : 0;
+  p.wcost = !p.inline_plan ? 0
+            : G <= 8       ? 0
+            : G <= 16      ? ETA_DECODE_PS_SEG_COST16
+                           : ETA_DECODE_PS_SEG_COST32;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = kDefaultWaitNs;
   const PsLayout L = ps_layout(B, Hkv, G, d, nc, !seg_aligned);

@@ -178,7 +178,8 @@ struct PParams {
   const void* vc;
   const int* seqlens;
   const long long* tok_off;  // [B]: token offset of sequence b in the packed cache
-  const int* tile_off;       // [B + 1]: first global tile of sequence b (all its KV heads)
+  const int* tile_off;       // [B + 1]: first global tile of sequence b (all its KV heads);
+                             // with wcost > 0 its first cost position (see wcost)
   void* o;                   // [B][Hq][D], input type (D = 64 or 128: the kernels' template)
   float* lse;                // [B][Hq] natural log, or NULL
   float* part_o;             // [slots][G][D]: normalised partial O of a cut segment
@@ -191,6 +192,8 @@ struct PParams {
   int window;       // > 0: each new token reads only the last `window` cached tokens
   int seg_aligned;  // 1: CTAs take whole segments (no partials); 0: equal tile ranges
   int inline_plan;  // 1: no plan kernel; each CTA finds its range from seqlens (equal ranges)
+  int wcost;        // inline plan only: each segment costs wcost tiles more than its own, and
+                    // the CTAs take equal shares of that cost (0: equal shares of the tiles)
   float scale_log2;
   uint64_t wait_ns;
 };
@@ -614,18 +617,27 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
   if (p.inline_plan) {
     // Prefix sums over the sequences in this CTA (small batches): the total
     // tile count, this CTA's range and its first tile, without a plan kernel.
-    // CTA 0 also writes the tile offsets the gather kernel reads, and CTA
-    // b % nc writes O = 0, LSE = -inf for an empty sequence b.
+    // Cost positions: each non-empty segment takes wcost positions, then one
+    // per tile; CTA c takes the tiles whose positions lie in
+    // [c C / nc, (c + 1) C / nc) of the C positions (wcost = 0: equal tile
+    // shares). CTA 0 also writes the sequences' first cost positions, which
+    // the gather kernel reads, and CTA b % nc writes O = 0, LSE = -inf for an
+    // empty sequence b. The token sums carry the count of non-empty sequences
+    // in their top 16 bits.
+    constexpr long long kSeqOne = 1ll << 48;
     long long* wsum = reinterpret_cast<long long*>(red);  // [warps][2], free before the stream
     volatile long long* start = reinterpret_cast<volatile long long*>(smem + C::kCtlOff + 40);
     const int nthr = R::kThreads, nw = nthr / 32;
+    volatile long long* ends = wsum + 2 * nw;  // [0]: the range's end tile, [1]: its first
     const int per = (p.B + nthr - 1) / nthr;
     const int b0 = threadIdx.x * per, b1 = min(p.B, b0 + per);
+    const int w = p.wcost;
     long long til = 0, tok = 0;
     for (int b = b0; b < b1; ++b) {
       const int len = max(p.seqlens[b], 0);
-      tok += len;
-      til += static_cast<long long>(p.Hkv) * ((len - first_key(len, p.window) + TK - 1) / TK);
+      const int nt = (len - first_key(len, p.window) + TK - 1) / TK;
+      tok += len + (nt > 0 ? kSeqOne : 0);
+      til += static_cast<long long>(p.Hkv) * nt;
     }
     long long xt = til, xk = tok;
 #pragma unroll
@@ -641,7 +653,10 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
       wsum[2 * warp] = xt;
       wsum[2 * warp + 1] = xk;
     }
-    if (threadIdx.x == 0) start[0] = -1;
+    if (threadIdx.x == 0) {
+      start[0] = -1;
+      ends[0] = -1;  // (no end found: all tiles)
+    }
     __syncthreads();
     if (warp == 0) {
       long long wt = lane < nw ? wsum[2 * lane] : 0, wk = lane < nw ? wsum[2 * lane + 1] : 0;
@@ -662,15 +677,20 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     }
     __syncthreads();
     const long long T_all = wsum[2 * (nw - 1)];
+    const long long wseg = static_cast<long long>(w) * p.Hkv;  // cost positions before a sequence's tiles
+    const long long C_all = T_all + wseg * (wsum[2 * (nw - 1) + 1] >> 48);
     long long l_run = xt - til + (warp > 0 ? wsum[2 * (warp - 1)] : 0);  // exclusive
     long long t_run = xk - tok + (warp > 0 ? wsum[2 * (warp - 1) + 1] : 0);
-    rg.lo = div_nonneg(c * T_all, gridDim.x);
-    rg.hi = div_nonneg((c + 1) * T_all, gridDim.x);
+    long long k_run = l_run + wseg * (t_run >> 48);
+    t_run &= kSeqOne - 1;
+    const long long x_lo = div_nonneg(c * C_all, gridDim.x);
+    const long long x_hi = div_nonneg((c + 1) * C_all, gridDim.x);
     for (int b = b0; b < b1; ++b) {
       const int len = max(p.seqlens[b], 0);
       const int nt = (len - first_key(len, p.window) + TK - 1) / TK;
       const long long span = static_cast<long long>(p.Hkv) * nt;
-      if (c == 0) const_cast<int*>(p.tile_off)[b] = static_cast<int>(l_run);
+      const long long kspan = nt > 0 ? span + wseg : 0;
+      if (c == 0) const_cast<int*>(p.tile_off)[b] = static_cast<int>(k_run);
       if (nt == 0 && b % static_cast<int>(gridDim.x) == c) {
         for (int h = 0; h < p.Hq; ++h) {
           const size_t row = static_cast<size_t>(b) * p.Hq + h;
@@ -679,17 +699,38 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
           if (p.lse != nullptr) p.lse[row] = -INFINITY;
         }
       }
-      if (rg.lo < rg.hi && l_run <= rg.lo && rg.lo < l_run + span) {
+      // The tile at or after cost position x of this sequence, as its rank
+      // g nt + i among the sequence's tiles (segment g, tile i; one of a
+      // segment's wcost leading positions gives its first tile). Segments
+      // are stepped over rather than divided: the start of the kernel is
+      // kept short (its instructions are fetched cold).
+      auto rank_at = [&](long long x) {
+        int r = static_cast<int>(x - k_run), g = 0;
+        while (r >= nt + w) {
+          r -= nt + w;
+          ++g;
+        }
+        return static_cast<long long>(g) * nt + max(r - w, 0);
+      };
+      if (k_run <= x_lo && x_lo < k_run + kspan) {
+        const long long rk = rank_at(x_lo);
         start[0] = b;
-        start[1] = rg.lo - l_run;
+        start[1] = rk;
         start[2] = t_run;
+        ends[1] = l_run + rk;
       }
+      if (k_run <= x_hi && x_hi < k_run + kspan) ends[0] = l_run + rank_at(x_hi);
       l_run += span;
+      k_run += kspan;
       t_run += len;
     }
-    if (c == 0 && threadIdx.x == 0) const_cast<int*>(p.tile_off)[p.B] = static_cast<int>(T_all);
+    if (c == 0 && threadIdx.x == 0) const_cast<int*>(p.tile_off)[p.B] = static_cast<int>(C_all);
     __syncthreads();
-    if (start[0] < 0) rg.hi = rg.lo;  // (no tile found: cannot happen when lo < T)
+    rg.lo = rg.hi = 0;  // no tiles at all
+    if (start[0] >= 0) {
+      rg.lo = ends[1];
+      rg.hi = ends[0] >= 0 ? ends[0] : T_all;
+    }
     if (rg.lo < rg.hi) {
       cur.b = static_cast<int>(start[0]);
       cur.load_seq(p);
@@ -1117,10 +1158,15 @@ __global__ void __launch_bounds__(128) attn_decode_gather_kernel(const PParams p
   const int h = static_cast<int>(row - static_cast<long long>(b) * p.Hq);
   const int g = h / p.G;
   const int hh = h - g * p.G;
-  const int nt = (p.tile_off[b + 1] - p.tile_off[b]) / p.Hkv;
-  if (nt == 0 || p.seg_aligned) return;
-  const long long T_all = p.tile_off[p.B];
-  const long long a = p.tile_off[b] + static_cast<long long>(g) * nt;
+  // tile_off holds cost positions (tile offsets when wcost = 0): a non-empty
+  // sequence spans Hkv (nt + wcost) of them, and tile i of its segment g sits
+  // at tile_off[b] + g (nt + wcost) + wcost + i.
+  const int w = p.wcost;
+  const int span = p.tile_off[b + 1] - p.tile_off[b];
+  if (span == 0 || p.seg_aligned) return;
+  const int nt = span / p.Hkv - w;
+  const long long T_all = p.tile_off[p.B];  // all cost positions
+  const long long a = p.tile_off[b] + static_cast<long long>(g) * (nt + w) + w;
   const int c0 = cta_of(a, T_all, nc);
   const int c1 = cta_of(a + nt - 1, T_all, nc);
   if (c0 == c1) return;
