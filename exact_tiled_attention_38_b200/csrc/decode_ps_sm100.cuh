@@ -554,6 +554,7 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
   // With the K/V split, full / empty track a stage's K tile and these its V tile.
   uint64_t* full_v = first_issued + 2;
   uint64_t* empty_v = full_v + kStages;
+  static_assert(sizeof(CtaCtl) <= 16, "control words, then the plan's range ends at +16");
   CtaCtl* ctl = reinterpret_cast<CtaCtl*>(smem + C::kCtlOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kCtlOff + 32);
 
@@ -628,7 +629,10 @@ __global__ void __launch_bounds__(Roles<HS>::kThreads, 1)
     long long* wsum = reinterpret_cast<long long*>(red);  // [warps][2], free before the stream
     volatile long long* start = reinterpret_cast<volatile long long*>(smem + C::kCtlOff + 40);
     const int nthr = R::kThreads, nw = nthr / 32;
-    volatile long long* ends = wsum + 2 * nw;  // [0]: the range's end tile, [1]: its first
+    // [0]: the range's end tile, [1]: its first; between the CTA's control
+    // words and the tensor-memory address (not in `red`, which the softmax
+    // warps take over once the stream runs).
+    volatile long long* ends = reinterpret_cast<volatile long long*>(smem + C::kCtlOff + 16);
     const int per = (p.B + nthr - 1) / nthr;
     const int b0 = threadIdx.x * per, b1 = min(p.B, b0 + per);
     const int w = p.wcost;
