@@ -6,8 +6,10 @@
 // Eliminating KV Cache"), so decode is a stream over the cache and its speed
 // is the rate at which each SM keeps that stream moving. The work is cut into
 // tiles of 128 keys of one (sequence b, KV head g) -- a "segment" -- and the
-// tiles of all segments, in order, are divided into equal contiguous ranges,
-// one per CTA (one CTA per SM). A CTA streams its range without a restart at
+// tiles of all segments, in order, are divided into contiguous ranges, one
+// per CTA (one CTA per SM): equal numbers of tiles, or, for groups above 8
+// in batches whose stream plans itself, equal shares of a cost that also
+// charges each segment start. A CTA streams its range without a restart at
 // segment boundaries: the K/V ring, the score products and the running
 // softmax (aikaboom page "11.4d FlashAttention", "Tiling" and "Online
 // Softmax") carry on, and at the end of each piece of a segment the CTA
@@ -24,6 +26,8 @@
 //                                  O = 0, LSE = -inf for empty sequences
 //   attn_decode_persistent_kernel  the stream (below); for smaller batches
 //                                  each CTA forms the same prefix sums itself
+//                                  (and the cost positions, which it records
+//                                  for the gather in place of tile offsets)
 //   attn_decode_gather_kernel      one warp per (sequence, query head) of a
 //                                  segment cut between CTAs: merges its
 //                                  partials by their log-sum-exp
@@ -191,7 +195,7 @@ struct PParams {
   int G;
   int window;       // > 0: each new token reads only the last `window` cached tokens
   int seg_aligned;  // 1: CTAs take whole segments (no partials); 0: equal tile ranges
-  int inline_plan;  // 1: no plan kernel; each CTA finds its range from seqlens (equal ranges)
+  int inline_plan;  // 1: no plan kernel; each CTA finds its range from seqlens itself
   int wcost;        // inline plan only: each segment costs wcost tiles more than its own, and
                     // the CTAs take equal shares of that cost (0: equal shares of the tiles)
   float scale_log2;
